@@ -1,0 +1,101 @@
+"""Pins of the oracle's block-sparse attention.
+
+Page: DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
+Generation, Methodology item 3 and Significance (block-wise execution over
+the kept blocks). A full mask is plain dense attention.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention, hilbert, pipeline, selection
+
+
+def _qkv(B, nh, N, D, seed=0):
+    r = np.random.default_rng(seed)
+    return [r.standard_normal((B, nh, N, D)) for _ in range(3)]
+
+
+def _full_lists(B, nh, nb):
+    idx = np.tile(np.arange(nb, dtype=np.int32), (B, nh, nb, 1))
+    cnt = np.full((B, nh, nb), nb, dtype=np.int32)
+    return idx, cnt
+
+
+def _loops_dense(q, k, v, scale):
+    """Softmax attention written with scalar loops and math.exp."""
+    N, D = q.shape
+    out = np.zeros((N, D))
+    for i in range(N):
+        logits = [scale * sum(q[i, d] * k[j, d] for d in range(D)) for j in range(N)]
+        m = max(logits)
+        e = [math.exp(x - m) for x in logits]
+        z = sum(e)
+        for d in range(D):
+            out[i, d] = sum(e[j] * v[j, d] for j in range(N)) / z
+    return out
+
+
+def test_dense_matches_scalar_loops():
+    q, k, v = _qkv(1, 1, 13, 4)
+    ref = _loops_dense(q[0, 0], k[0, 0], v[0, 0], 0.5)
+    got = attention.dense_attention(q, k, v, 0.5)[0, 0]
+    assert np.abs(got - ref).max() < 1e-12
+
+
+def test_full_mask_is_dense():
+    B, nh, N, D, blk = 1, 2, 37, 8, 8
+    q, k, v = _qkv(B, nh, N, D, 1)
+    nb = -(-N // blk)
+    idx, cnt = _full_lists(B, nh, nb)
+    o, lse = attention.block_sparse_attention(q, k, v, idx, cnt, blk)
+    assert np.abs(o - attention.dense_attention(q, k, v)).max() < 1e-12
+    s = np.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(D)
+    assert np.abs(lse - np.log(np.exp(s).sum(-1))).max() < 1e-12
+
+
+def test_diagonal_mask_is_local_attention():
+    B, nh, N, D, blk = 1, 1, 20, 4, 8
+    q, k, v = _qkv(B, nh, N, D, 2)
+    nb = -(-N // blk)
+    idx = np.arange(nb, dtype=np.int32).reshape(1, 1, nb, 1)
+    cnt = np.ones((1, 1, nb), dtype=np.int32)
+    o, _ = attention.block_sparse_attention(q, k, v, idx, cnt, blk, 0.7)
+    for I in range(nb):
+        lo, hi = I * blk, min(N, I * blk + blk)
+        ref = _loops_dense(q[0, 0, lo:hi], k[0, 0, lo:hi], v[0, 0, lo:hi], 0.7)
+        assert np.abs(o[0, 0, lo:hi] - ref).max() < 1e-12
+
+
+def test_constant_v_gives_constant_output():
+    B, nh, N, D, blk = 1, 1, 30, 4, 8
+    q, k, _ = _qkv(B, nh, N, D, 3)
+    v = np.ones((B, nh, N, D)) * np.array([1.5, -2.0, 0.25, 7.0])
+    s = np.random.default_rng(3).standard_normal((B, nh, 4, 4))
+    idx, cnt = selection.select(s, "topk", k=2)
+    o, _ = attention.block_sparse_attention(q, k, v, idx, cnt, blk)
+    assert np.abs(o - v).max() < 1e-12
+
+
+def test_empty_list_gives_zero():
+    q, k, v = _qkv(1, 1, 16, 4, 4)
+    idx = np.full((1, 1, 2, 2), -1, dtype=np.int32)
+    cnt = np.array([[[0, 1]]], dtype=np.int32)
+    idx[0, 0, 1, 0] = 0
+    o, lse = attention.block_sparse_attention(q, k, v, idx, cnt, 8)
+    assert (o[0, 0, :8] == 0).all() and np.isneginf(lse[0, 0, :8]).all()
+    assert np.isfinite(o[0, 0, 8:]).all()
+
+
+def test_pipeline_tiny_grid_full_keep_is_dense():
+    # end to end: Hilbert reorder, scoring, top-k with k = nb, attention,
+    # inverse reorder equals dense attention in the raster order
+    T, H, W, nh, D = 2, 4, 4, 2, 8
+    N = T * H * W
+    r = np.random.default_rng(5)
+    q, k, v = (r.standard_normal((1, N, nh, D)) for _ in range(3))
+    res = pipeline.run(q, k, v, T=T, H=H, W=W, blk=8, sb=4, order="hilbert3d",
+                       mode="topk", k_keep=4)
+    dense = attention.dense_attention(*(np.transpose(x, (0, 2, 1, 3)) for x in (q, k, v)))
+    assert np.abs(res["out"] - np.transpose(dense, (0, 2, 1, 3))).max() < 1e-12
