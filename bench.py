@@ -1,0 +1,401 @@
+"""Benchmark of the DFSAttn hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = the whole path over one layer's synthetic Q/K/V already in HBM:
+Hilbert gather of Q, K, V -> pooled sub-block scoring -> top-k / threshold /
+LVSA selection -> block-sparse attention -> inverse gather. The curve index
+is built once per grid shape before timing (it depends only on the shape).
+Metric: kept-block TFLOP/s of the whole step (4 * D FLOPs per kept, valid
+query-key pair), with ms per step; the roofline object reports the
+attention kernel alone against the measured bf16 tensor peak.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own
+independent layer (weak scaling, no collective on the data path); the time
+is the maximum over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this
+method has) on the host cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
+KERNELS_PER_STEP = {"topk": 8, "threshold": 8, "lvsa": 6}   # 3 gathers, pool, score, select, attn, scatter
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(wl, k, cap):
+    sel = {"topk": f"top-k {k}/{wl.nb}", "threshold": f"threshold tau={wl.tau} cap {cap}/{wl.nb}",
+           "lvsa": f"LVSA T_per={wl.lvsa_T_per} C={wl.lvsa_C} step {wl.lvsa_step}"}[wl.mode]
+    return (f"{wl.name}: B={wl.B} nh={wl.nh} D={wl.D} grid {wl.T}x{wl.H}x{wl.W} (N={wl.N}) "
+            f"{wl.order} order, blk {wl.blk}, sb {wl.sb}, {sel}")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def make_layer(bsa, wl):
+    s = bsa.Shape(wl.B, wl.nh, wl.D, wl.T, wl.H, wl.W, wl.blk, wl.sb)
+    k = cap = 0
+    if wl.mode == "topk":
+        k = wl.ratio_count(wl.keep_num)
+        layer = bsa.DfsLayer(s, order=wl.order, mode="topk", k=k)
+    elif wl.mode == "threshold":
+        cap = wl.ratio_count(wl.cap_num)
+        layer = bsa.DfsLayer(s, order=wl.order, mode="threshold", cap=cap, tau=wl.tau)
+    else:
+        layer = bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
+                             lvsa_step=wl.lvsa_step)
+    return layer, k, cap
+
+
+def run_ours(args):
+    import torch
+    import synth
+    import block_sparse_attention_36_b200 as bsa
+    from block_sparse_attention_36_b200 import dfsattn
+
+    rank, world, local = dist_setup(args.gpus)
+    wl = synth.WORKLOADS[args.workload]
+    if wl.mode == "schedule":
+        raise SystemExit("the schedule workload is timed by --workload wan_schedule_50 via run_schedule")
+    qkv = synth.workload_inputs(wl, seed=args.seed + rank)
+    q, k, v = (qkv[n].cuda() for n in ("q", "k", "v"))
+    layer, kk, cap = make_layer(bsa, wl)
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also builds the curve index once)
+    for _ in range(args.warmup):
+        layer.forward(q, k, v)
+    torch.cuda.synchronize()
+    kept_pairs = layer.kept_pairs()
+    flops_step = 4.0 * wl.D * kept_pairs * 1.0
+    dense_flops = 4.0 * wl.D * wl.N * wl.N * wl.nh * wl.B
+    assert dfsattn.dfs_get_error_flags(clear=True) == 0
+
+    # timed region: K whole steps; attention kernel bracketed by its own events
+    ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        layer.permute(q, k, v)
+        layer.build_mask()
+        ev_attn[i][0].record(stream)
+        dfsattn.dfs_sparse_attn_fwd(layer.shape, layer.qp, layer.kp, layer.vp, layer.kv_idx, layer.kv_cnt,
+                                    layer.kcap, layer.scale, layer.op, None)
+        ev_attn[i][1].record(stream)
+        dfsattn.dfs_unperm(layer.shape, layer.perm, layer.op, layer.out)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    ms_total = start.elapsed_time(stop)
+    attn_ms = [a.elapsed_time(b) for a, b in ev_attn]
+    ms_total_max = max_over_ranks(ms_total, world)
+    flops_all = sum_over_ranks(flops_step * args.steps, world)
+    attn_avg = statistics.mean(attn_ms)
+
+    # end to end through the C ABI from pinned host buffers
+    hq, hk, hv = (qkv[n].pin_memory() for n in ("q", "k", "v"))
+    ho = torch.empty_like(hq).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        layer.forward(q, k, v)
+        ho.copy_(layer.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        layer.forward(q, k, v)
+        ho.copy_(layer.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e_flops = sum_over_ranks(flops_step, world)
+    assert dfsattn.dfs_get_error_flags(clear=True) == 0
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        achieved = flops_step / (attn_avg * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        ms_step = ms_total_max / args.steps
+        value = flops_all / (ms_total_max * 1e-3) / 1e12
+        traffic = None
+        line = {
+            "metric": METRIC,
+            "value": round(value, 3),
+            "unit": "TFLOP/s (kept-block, whole step)",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4),
+            "attn_ms_per_call": round(attn_avg, 4),
+            "dense_equiv_tflops": round(dense_flops / (ms_step * 1e-3) / 1e12, 3),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded smooth Fourier field + noise, bf16)",
+            "config": {"workload": workload_config(wl, kk, cap), "kept_pairs_per_step": kept_pairs,
+                       "kept_fraction": round(kept_pairs / (wl.N * wl.N * wl.nh * wl.B), 4),
+                       "l2": "inputs larger than L2 (3 x %.1f MB of Q/K/V per step)" % (wl.N * wl.nh * wl.D * 2 / 1e6),
+                       "parallelism": f"replicas x{world} (independent layer per GPU)"},
+            "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(achieved, 2),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "peak_source": f"{src} bf16 burst", "traffic": traffic},
+            "e2e": {"value": round(e2e_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s (kept-block, whole step)",
+                    "ms_per_step": round(e2e_ms, 3),
+                    "h2d_bytes_per_step": int(3 * hq.numel() * hq.element_size()),
+                    "d2h_bytes_per_step": int(ho.numel() * ho.element_size())},
+            "gpu_launches": KERNELS_PER_STEP[wl.mode] * args.steps,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(wl, qkv, kk, cap, budget_s=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, steps=1):
+    """Times the oracle on the host over a bounded sample of the workload.
+
+    The sample: the curve index, scoring and selection over the whole layer,
+    then attention on as many randomly chosen query blocks as fit the time
+    budget; the time per query block is scaled to the whole layer.
+    Returns the oracle's whole-step throughput in the same unit."""
+    import torch
+    from oracle import attention, hilbert, lvsa, scoring, selection
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    t0 = time.perf_counter()
+    perm, _ = hilbert.make_perm(wl.order, wl.T, wl.H, wl.W)
+    permt = torch.from_numpy(perm.astype(np.int64))
+    t_perm = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    t_mask = 0.0
+    t_attn = 0.0
+    n_rows = 0
+    kept = 0
+    per_head = []
+    for h in range(wl.nh):
+        t1 = time.perf_counter()
+        qp, kp, vp = (qkv[n][0, permt, h, :].double().numpy()[None, None] for n in ("q", "k", "v"))
+        if wl.mode == "lvsa":
+            m = lvsa.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step) if h == 0 else m
+            idx, cnt = selection.mask_to_lists(m[None, None])
+        else:
+            sc = scoring.block_scores(qp, kp, wl.blk, wl.sb)
+            idx, cnt = selection.select(sc, wl.mode, k=k, tau=wl.tau, cap=cap)
+        t_mask += time.perf_counter() - t1
+        per_head.append((qp, kp, vp, idx, cnt))
+        if time.perf_counter() - t0 > budget_s * 0.6 and h < wl.nh - 1:
+            # scoring of the remaining heads is estimated from the mean so far
+            t_mask = t_mask / (h + 1) * wl.nh
+            break
+    heads_done = len(per_head)
+    deadline = time.perf_counter() + max(1.0, budget_s - (time.perf_counter() - t0))
+    rows_total = wl.nb * wl.nh * wl.B
+    while time.perf_counter() < deadline:
+        h = int(rng.integers(0, heads_done))
+        I = int(rng.integers(0, wl.nb))
+        qp, kp, vp, idx, cnt = per_head[h]
+        t1 = time.perf_counter()
+        attention.block_sparse_attention(qp, kp, vp, idx, cnt, wl.blk, rows=[(0, 0, I)])
+        t_attn += time.perf_counter() - t1
+        n_rows += 1
+        rows_q = min(wl.blk, wl.N - I * wl.blk)
+        c = int(cnt[0, 0, I])
+        js = idx[0, 0, I, :c]
+        kept += rows_q * int(sum(min(wl.blk, wl.N - j * wl.blk) for j in js))
+    t_attn_full = t_attn / max(1, n_rows) * rows_total
+    t_step = t_perm + t_mask + t_attn_full
+    kept_full = kept / max(1, n_rows) * rows_total
+    flops = 4.0 * wl.D * kept_full
+    return {"value": round(flops / t_step / 1e12, 6), "unit": "TFLOP/s (kept-block, whole step)",
+            "cores": threads, "kind": "oracle",
+            "ms_per_step": round(t_step * 1e3, 1),
+            "sample": (f"curve index; scoring+selection on {heads_done}/{wl.nh} heads (rest scaled); "
+                       f"fp64 attention on {n_rows} random query blocks of {rows_total} (scaled)")}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    qkv = synth.workload_inputs(wl, seed=args.seed)
+    k = wl.ratio_count(wl.keep_num) if wl.mode == "topk" else 0
+    cap = wl.ratio_count(wl.cap_num) if wl.mode == "threshold" else 0
+    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(wl, qkv, k, cap, budget_s=budget / 4)
+    vals = [cpu_baseline(wl, qkv, k, cap, budget_s=budget) for _ in range(args.steps)]
+    ms = statistics.mean(v["ms_per_step"] for v in vals)
+    val = statistics.mean(v["value"] for v in vals)
+    unit = vals[0]["unit"]
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_config(wl, k, cap), "parallelism": "host cores, rank 0 only"},
+            "cpu_baseline": {"value": round(val, 6), "unit": unit, "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": round(val, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="wan_1p3b_layer")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,253 @@
+// Token reorder along the global 3D Hilbert curve and its inverse.
+//
+// DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
+// Generation, Methodology item 1: tokens are reordered along one global 3D
+// Hilbert curve before attention, keeping spatiotemporal neighbours close
+// and memory access contiguous.
+//
+// Curve: the generalised Hilbert curve of an arbitrary box, built by
+// recursive splitting (the published "gilbert" construction). A box is an
+// entry cell p plus three orthogonal axis-parallel vectors a (major), b, c;
+// its path starts at p and ends one step short of p + a. Boxes with two unit
+// sides are walked straight; otherwise the sides are halved (rounded toward
+// zero, then made even when the side exceeds 2) and the box is cut into 2,
+// 3 or 5 sub-boxes depending on its aspect ratio (wide: 2w > 3h and 2w > 3d;
+// tall: 3h > 4d; deep: 3d > 4h; else regular). Here each thread finds the
+// cell of one curve rank by descending into the sub-box that holds it, so
+// the index kernel needs no traversal and no scratch memory.
+//
+// Gather / scatter: 16-byte vector loads and stores. A token-major row of
+// nh*D bf16 values is contiguous in the raster layout; a head's D values of
+// consecutive curve positions are contiguous in the head-major layout, so
+// both sides move whole 256-byte (D = 128) or 128-byte (D = 64) runs.
+#include "common.cuh"
+
+namespace {
+
+__device__ uint32_t g_perm_flags;
+
+// An axis-parallel vector: coordinate index (0 = t, 1 = h, 2 = w) and signed
+// length along it.
+struct Axis {
+  int dim;
+  int len;
+};
+
+__device__ __forceinline__ int alen(Axis a) { return a.len < 0 ? -a.len : a.len; }
+__device__ __forceinline__ int asign(Axis a) { return a.len < 0 ? -1 : 1; }
+__device__ __forceinline__ Axis aneg(Axis a) { return Axis{a.dim, -a.len}; }
+// a - b for parallel a, b.
+__device__ __forceinline__ Axis aminus(Axis a, Axis b) { return Axis{a.dim, a.len - b.len}; }
+// a shortened by one unit step (the vector to its last cell).
+__device__ __forceinline__ Axis alast(Axis a) { return Axis{a.dim, a.len - asign(a)}; }
+__device__ __forceinline__ Axis ahalf(Axis a) {
+  int n = alen(a);
+  int h = n >> 1;
+  if ((h & 1) && n > 2) ++h;
+  return Axis{a.dim, a.len < 0 ? -h : h};
+}
+
+struct Box {
+  int p[3];
+  Axis a, b, c;
+};
+
+__device__ __forceinline__ long long box_volume(const Box& x) {
+  return (long long)alen(x.a) * alen(x.b) * alen(x.c);
+}
+
+__device__ __forceinline__ void shift(int p[3], Axis v) { p[v.dim] += v.len; }
+
+__device__ __forceinline__ Box make_box(const int p[3], Axis o1, Axis o2, Axis o3,
+                                        Axis a, Axis b, Axis c) {
+  Box x;
+  x.p[0] = p[0]; x.p[1] = p[1]; x.p[2] = p[2];
+  shift(x.p, o1); shift(x.p, o2); shift(x.p, o3);
+  x.a = a; x.b = b; x.c = c;
+  return x;
+}
+
+// Cell (t, h, w) at rank r of the curve over box `top`.
+__device__ void hilbert_cell(Box cur, long long r, int out[3]) {
+  const Axis zero{0, 0};
+  for (int guard = 0; guard < 256; ++guard) {
+    const int w = alen(cur.a), h = alen(cur.b), d = alen(cur.c);
+    if (h == 1 && d == 1) { cur.p[cur.a.dim] += asign(cur.a) * (int)r; break; }
+    if (w == 1 && d == 1) { cur.p[cur.b.dim] += asign(cur.b) * (int)r; break; }
+    if (w == 1 && h == 1) { cur.p[cur.c.dim] += asign(cur.c) * (int)r; break; }
+    const Axis a2 = ahalf(cur.a), b2 = ahalf(cur.b), c2 = ahalf(cur.c);
+    Box kids[5];
+    int nk;
+    if (2 * w > 3 * h && 2 * w > 3 * d) {
+      kids[0] = make_box(cur.p, zero, zero, zero, a2, cur.b, cur.c);
+      kids[1] = make_box(cur.p, a2, zero, zero, aminus(cur.a, a2), cur.b, cur.c);
+      nk = 2;
+    } else if (3 * h > 4 * d) {
+      kids[0] = make_box(cur.p, zero, zero, zero, b2, cur.c, a2);
+      kids[1] = make_box(cur.p, b2, zero, zero, cur.a, aminus(cur.b, b2), cur.c);
+      kids[2] = make_box(cur.p, alast(cur.a), alast(b2), zero, aneg(b2), cur.c,
+                         aneg(aminus(cur.a, a2)));
+      nk = 3;
+    } else if (3 * d > 4 * h) {
+      kids[0] = make_box(cur.p, zero, zero, zero, c2, a2, cur.b);
+      kids[1] = make_box(cur.p, c2, zero, zero, cur.a, cur.b, aminus(cur.c, c2));
+      kids[2] = make_box(cur.p, alast(cur.a), alast(c2), zero, aneg(c2),
+                         aneg(aminus(cur.a, a2)), cur.b);
+      nk = 3;
+    } else {
+      kids[0] = make_box(cur.p, zero, zero, zero, b2, c2, a2);
+      kids[1] = make_box(cur.p, b2, zero, zero, cur.c, a2, aminus(cur.b, b2));
+      kids[2] = make_box(cur.p, alast(b2), alast(cur.c), zero, cur.a, aneg(b2),
+                         aneg(aminus(cur.c, c2)));
+      kids[3] = make_box(cur.p, alast(cur.a), b2, alast(cur.c), aneg(cur.c),
+                         aneg(aminus(cur.a, a2)), aminus(cur.b, b2));
+      kids[4] = make_box(cur.p, alast(cur.a), alast(b2), zero, aneg(b2), c2,
+                         aneg(aminus(cur.a, a2)));
+      nk = 5;
+    }
+    int pick = nk - 1;
+    for (int i = 0; i < nk; ++i) {
+      const long long v = box_volume(kids[i]);
+      if (r < v) { pick = i; break; }
+      r -= v;
+    }
+    cur = kids[pick];
+  }
+  out[0] = cur.p[0]; out[1] = cur.p[1]; out[2] = cur.p[2];
+}
+
+__global__ void hilbert_index_kernel(int T, int H, int W, int order, int32_t* __restrict__ perm,
+                                     int32_t* __restrict__ inv) {
+  const long long N = (long long)T * H * W;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  long long n;
+  if (order == DFS_ORDER_RASTER) {
+    n = i;
+  } else {
+    // Major axis: the longest side, ties to W, then H, then T; the other two
+    // in the order W, H, T.
+    Axis aw{2, W}, ah{1, H}, at{0, T};
+    Box top;
+    top.p[0] = top.p[1] = top.p[2] = 0;
+    if (W >= H && W >= T) { top.a = aw; top.b = ah; top.c = at; }
+    else if (H >= T) { top.a = ah; top.b = aw; top.c = at; }
+    else { top.a = at; top.b = aw; top.c = ah; }
+    int cell[3];
+    hilbert_cell(top, i, cell);
+    n = ((long long)cell[0] * H + cell[1]) * W + cell[2];
+    if (cell[0] < 0 || cell[0] >= T || cell[1] < 0 || cell[1] >= H || cell[2] < 0 || cell[2] >= W)
+      n = 0;  // unreachable for valid shapes; keeps the write in bounds
+  }
+  perm[i] = (int32_t)n;
+  inv[n] = (int32_t)i;
+}
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 8;
+
+// Moves 16-byte vectors between the token-major layout [B, N, nh*D] and the
+// head-major layout [B, nh, N, D] through perm.
+//   to_curve = true : dst_headmajor[b, h, i, :] = src_tokmajor[b, perm[i], h, :]
+//   to_curve = false: dst_tokmajor[b, perm[i], h, :] = src_headmajor[b, h, i, :]
+// The flat work index e runs over (b, i, vec) with vec = h * (D/8) + d8
+// (e < 2^31, checked on the host); each thread handles kCopyUnroll vectors
+// spaced kCopyThreads apart and issues all its loads before its stores.
+template <bool kToCurve>
+__global__ void __launch_bounds__(kCopyThreads)
+permute_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                    const int32_t* __restrict__ perm, uint32_t N, uint32_t nh, uint32_t dvec,
+                    dfs::FastDiv div_vpt, dfs::FastDiv div_n, dfs::FastDiv div_dvec,
+                    uint32_t total) {
+  const uint32_t vpt = nh * dvec;  // vectors per token
+  const uint32_t base = blockIdx.x * (kCopyThreads * kCopyUnroll) + threadIdx.x;
+  uint4 val[kCopyUnroll];
+  long long dst_off[kCopyUnroll];
+#pragma unroll
+  for (int u = 0; u < kCopyUnroll; ++u) {
+    const uint32_t e = base + (uint32_t)u * kCopyThreads;
+    dst_off[u] = -1;
+    if (e < total) {
+      const uint32_t tok = div_vpt.div(e);      // flat (b, i)
+      const uint32_t vec = e - tok * vpt;
+      const uint32_t b = div_n.div(tok);
+      const uint32_t i = tok - b * N;
+      const uint32_t h = div_dvec.div(vec);
+      const uint32_t d8 = vec - h * dvec;
+      const long long n = perm[i];
+      const long long tokmajor = ((long long)b * N + n) * vpt + vec;
+      const long long headmajor = (((long long)b * nh + h) * N + i) * dvec + d8;
+      if (kToCurve) {
+        val[u] = __ldg(src + tokmajor);
+        dst_off[u] = headmajor;
+      } else {
+        val[u] = __ldg(src + headmajor);
+        dst_off[u] = tokmajor;
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kCopyUnroll; ++u)
+    if (dst_off[u] >= 0) dst[dst_off[u]] = val[u];
+}
+
+int launch_copy(bool to_curve, const void* src, void* dst, const int32_t* perm, const dfs::Dims& d,
+                cudaStream_t st) {
+  const int dvec = d.D / 8;
+  const long long total = (long long)d.B * d.N * d.nh * dvec;
+  if (total >= (1LL << 31)) return DFS_ERR_UNSUPPORTED;
+  const long long per_block = (long long)kCopyThreads * kCopyUnroll;
+  const unsigned grid = (unsigned)((total + per_block - 1) / per_block);
+  const dfs::FastDiv dv((uint32_t)(d.nh * dvec)), dn((uint32_t)d.N), dd((uint32_t)dvec);
+  if (to_curve)
+    permute_copy_kernel<true><<<grid, kCopyThreads, 0, st>>>(
+        (const uint4*)src, (uint4*)dst, perm, (uint32_t)d.N, d.nh, dvec, dv, dn, dd, (uint32_t)total);
+  else
+    permute_copy_kernel<false><<<grid, kCopyThreads, 0, st>>>(
+        (const uint4*)src, (uint4*)dst, perm, (uint32_t)d.N, d.nh, dvec, dv, dn, dd, (uint32_t)total);
+  return dfs::launch_status();
+}
+
+}  // namespace
+
+DFS_DEFINE_FLAG_READER(dfs_detail_flags_perm, g_perm_flags)
+
+extern "C" int dfs_hilbert_perm(const dfs_shape* shape, int order, int32_t* perm, int32_t* inv,
+                                int build_index, const void* q, const void* k, const void* v,
+                                void* qp, void* kp, void* vp, dfs_stream_t stream) {
+  dfs::Dims d;
+  int st = dfs::check_shape(shape, &d, false);
+  if (st != DFS_OK) return st;
+  if (order != DFS_ORDER_RASTER && order != DFS_ORDER_HILBERT3D) return DFS_ERR_INVALID_ARG;
+  if (!perm || (build_index && !inv)) return DFS_ERR_INVALID_ARG;
+  const void* srcs[3] = {q, k, v};
+  void* dsts[3] = {qp, kp, vp};
+  for (int t = 0; t < 3; ++t) {
+    if ((srcs[t] == nullptr) != (dsts[t] == nullptr)) return DFS_ERR_INVALID_ARG;
+    if (srcs[t] && (!dfs::aligned16(srcs[t]) || !dfs::aligned16(dsts[t]))) return DFS_ERR_MISALIGNED;
+  }
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (build_index) {
+    const int threads = 256;
+    const long long grid = (d.N + threads - 1) / threads;
+    hilbert_index_kernel<<<(unsigned)grid, threads, 0, cs>>>(d.T, d.H, d.W, order, perm, inv);
+    st = dfs::launch_status();
+    if (st != DFS_OK) return st;
+  }
+  for (int t = 0; t < 3; ++t) {
+    if (!srcs[t]) continue;
+    st = launch_copy(true, srcs[t], dsts[t], perm, d, cs);
+    if (st != DFS_OK) return st;
+  }
+  return DFS_OK;
+}
+
+extern "C" int dfs_unperm(const dfs_shape* shape, const int32_t* perm, const void* op, void* o,
+                          dfs_stream_t stream) {
+  dfs::Dims d;
+  int st = dfs::check_shape(shape, &d, false);
+  if (st != DFS_OK) return st;
+  if (!perm || !op || !o) return DFS_ERR_INVALID_ARG;
+  if (!dfs::aligned16(op) || !dfs::aligned16(o)) return DFS_ERR_MISALIGNED;
+  return launch_copy(false, op, o, perm, d, (cudaStream_t)stream);
+}

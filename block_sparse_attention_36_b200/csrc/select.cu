@@ -1,0 +1,286 @@
+// Per-query-block key-block selection.
+//
+//  * top-k -- DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient
+//    Video Generation, Methodology item 3 (a sparsity budget per query
+//    block): the k highest scores of the row, equal scores to the lower
+//    block index.
+//  * threshold -- VMoBA: Mixture of Block Attention for Video Diffusion
+//    Models, abstract, modification (3): p = softmax of the row; the fewest
+//    best-ranked blocks whose mass reaches tau, at most cap.
+//  * LVSA -- LVSA: Training-Free Sparse Attention for Long Video Diffusion,
+//    section 2: rotating global anchors plus an expanded local window of
+//    frames, mapped onto key blocks.
+//
+// One warp per row. Scores live in registers, lane l holding columns
+// l, l + 32, l + 64, ... Scores map to order-preserving 32-bit keys; the
+// k-th largest key comes from a 32-step bitwise descent with warp-wide
+// counts (__reduce_add_sync), the threshold cut from the same descent on
+// warp-wide mass sums. Kept columns are emitted in ascending order with
+// ballots and popcounts; equal keys at the cut go to the lowest columns.
+#include "common.cuh"
+
+namespace {
+
+__device__ uint32_t g_select_flags;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  f = f + 0.0f;  // -0 -> +0, so equal values compare equal
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Largest key value K with count(key >= K) >= k (k >= 1, k <= n).
+template <int S>
+__device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&key)[S], const bool (&valid)[S], int k) {
+  uint32_t K = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = K | (1u << bit);
+    uint32_t c = 0;
+#pragma unroll
+    for (int s = 0; s < S; ++s) c += (valid[s] && key[s] >= cand) ? 1u : 0u;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= (uint32_t)k) K = cand;
+  }
+  return K;
+}
+
+// Writes the kept columns of a row in ascending order: every column with
+// key > K, plus the first `ties` columns with key == K.
+template <int S>
+__device__ __forceinline__ int emit_row(const uint32_t (&key)[S], const bool (&valid)[S], uint32_t K,
+                                        int ties, int32_t* out, int kcap, int lane) {
+  int base = 0, tie_seen = 0;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const bool gt = valid[s] && key[s] > K;
+    const bool eq = valid[s] && key[s] == K;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool take_eq = eq && (tie_seen + __popc(eqb & lt)) < ties;
+    tie_seen += __popc(eqb);
+    const bool take = gt || take_eq;
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = base + __popc(tb & lt);
+    if (take && pos < kcap) out[pos] = s * 32 + lane;
+    base += __popc(tb);
+  }
+  return base;
+}
+
+template <int S>
+__global__ void __launch_bounds__(256)
+select_scores_kernel(const float* __restrict__ scores, int rows, int nb, int mode, int k, int cap,
+                     float tau, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, int kcap) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float* src = scores + row * nb;
+  float sc[S];
+  uint32_t key[S];
+  bool valid[S];
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int j = s * 32 + lane;
+    valid[s] = j < nb;
+    sc[s] = valid[s] ? __ldg(src + j) : -INFINITY;
+    key[s] = valid[s] ? order_key(sc[s]) : 0u;
+  }
+  int32_t* out = kv_idx + row * (long long)kcap;
+  int kept;
+  uint32_t K;
+  int ties;
+  int take = 0;  // number of blocks to keep
+  if (mode == DFS_SEL_TOPK) {
+    take = min(k, nb);
+  } else {
+    // threshold: smallest best-ranked prefix with mass >= tau * Z
+    float m = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < S; ++s) m = fmaxf(m, sc[s]);
+    m = warp_max(m);
+    float p[S];
+    float z = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      p[s] = valid[s] ? expf(sc[s] - m) : 0.f;
+      z += p[s];
+    }
+    z = warp_sum(z);
+    const float target = tau * z;
+    // Largest key value K with mass(key >= K) >= target.
+    uint32_t KK = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = KK | (1u << bit);
+      float ms = 0.f;
+#pragma unroll
+      for (int s = 0; s < S; ++s) ms += (valid[s] && key[s] >= cand) ? p[s] : 0.f;
+      ms = warp_sum(ms);
+      if (ms >= target) KK = cand;
+    }
+    // Blocks strictly above the cut, their mass, and the tie value at the cut.
+    uint32_t cgt = 0, ceq = 0;
+    float mgt = 0.f, peq = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      if (valid[s] && key[s] > KK) { cgt++; mgt += p[s]; }
+      if (valid[s] && key[s] == KK) { ceq++; peq = p[s]; }
+    }
+    cgt = __reduce_add_sync(0xffffffffu, cgt);
+    ceq = __reduce_add_sync(0xffffffffu, ceq);
+    mgt = warp_sum(mgt);
+    peq = warp_max(peq);
+    // mgt < target by the choice of KK (the warp sums are monotone in the
+    // set summed). Equal scores carry equal mass: add them one at a time,
+    // lowest column first, until the target is reached.
+    int t = 0;
+    float acc = mgt;
+    while (t < (int)ceq && acc < target) { acc += peq; ++t; }
+    take = max(1, (int)cgt + t);   // the shortest prefix holds at least one block
+    take = min(take, min(cap, nb));
+  }
+  if (take <= 0) {
+    kept = 0;
+  } else if (take >= nb) {
+    // keep all columns
+    K = 0u;
+    ties = nb;
+    bool all[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) all[s] = valid[s];
+    uint32_t zk[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) zk[s] = 0u;
+    kept = emit_row<S>(zk, all, K, ties, out, kcap, lane);
+  } else {
+    K = kth_largest_key<S>(key, valid, take);
+    uint32_t cgt = 0;
+#pragma unroll
+    for (int s = 0; s < S; ++s) cgt += (valid[s] && key[s] > K) ? 1u : 0u;
+    cgt = __reduce_add_sync(0xffffffffu, cgt);
+    ties = take - (int)cgt;
+    kept = emit_row<S>(key, valid, K, ties, out, kcap, lane);
+  }
+  if (lane == 0) {
+    if (kept > kcap) atomicOr(&g_select_flags, (uint32_t)DFS_FLAG_KCAP_OVERFLOW);
+    kv_cnt[row] = min(kept, kcap);
+  }
+}
+
+// Number of anchor frames in [lo, hi] (anchors: f mod T_per == s0).
+__device__ __forceinline__ int anchors_in(int lo, int hi, int T_per, int s0) {
+  if (hi < lo) return 0;
+  // count of f in [lo, hi] with f = s0 + m * T_per, m integer
+  auto fl = [](int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); };
+  return fl(hi - s0, T_per) - fl(lo - 1 - s0, T_per);
+}
+
+// Is frame f in A(t)? Anchors always; otherwise f must be among the
+// (C - |G|) non-anchor frames nearest to t in the scan order
+// t, t-1, t+1, t-2, t+2, ... (frames outside [0, T) skipped).
+__device__ __forceinline__ bool in_frame_set(int f, int t, int T, int T_per, int s0, int C, int nG) {
+  if (((f - s0) % T_per + T_per) % T_per == 0) return true;
+  const int need = C - nG;
+  if (need <= 0) return false;
+  const int dist = f > t ? f - t : t - f;
+  // non-anchor frames scanned before f: all of (t-dist, t+dist) ...
+  int lo = max(0, t - dist + 1), hi = min(T - 1, t + dist - 1);
+  int before = (hi >= lo) ? (hi - lo + 1) - anchors_in(lo, hi, T_per, s0) : 0;
+  // ... plus t - dist when f = t + dist (the earlier side goes first)
+  if (dist > 0 && f > t) {
+    const int g = t - dist;
+    if (g >= 0 && ((g - s0) % T_per + T_per) % T_per != 0) ++before;
+  }
+  return before < need;
+}
+
+__global__ void __launch_bounds__(256)
+select_lvsa_kernel(int rows, int nb, long long N, int blk, int P, int T, int T_per, int C, int s0,
+                   int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, int kcap) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int I = (int)(row % nb);
+  const int nG = (s0 < T) ? (T - 1 - s0) / T_per + 1 : 0;
+  const int qf0 = (int)(((long long)I * blk) / P);
+  const int qf1 = (int)((min((long long)I * blk + blk, N) - 1) / P);
+  int32_t* out = kv_idx + row * (long long)kcap;
+  const unsigned lt = (1u << lane) - 1u;
+  int base = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int J = j0 + lane;
+    bool take = false;
+    if (J < nb) {
+      const int kf0 = (int)(((long long)J * blk) / P);
+      const int kf1 = (int)((min((long long)J * blk + blk, N) - 1) / P);
+      for (int f = kf0; f <= kf1 && !take; ++f)
+        for (int t = qf0; t <= qf1 && !take; ++t)
+          take = in_frame_set(f, t, T, T_per, s0, C, nG);
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = base + __popc(tb & lt);
+    if (take && pos < kcap) out[pos] = J;
+    base += __popc(tb);
+  }
+  if (lane == 0) {
+    if (base > kcap) atomicOr(&g_select_flags, (uint32_t)DFS_FLAG_KCAP_OVERFLOW);
+    kv_cnt[row] = min(base, kcap);
+  }
+}
+
+}  // namespace
+
+DFS_DEFINE_FLAG_READER(dfs_detail_flags_select, g_select_flags)
+
+extern "C" int dfs_select_mask(const dfs_shape* shape, const float* scores, const dfs_select_params* prm,
+                               int32_t* kv_idx, int32_t* kv_cnt, int kcap, dfs_stream_t stream) {
+  dfs::Dims d;
+  int st = dfs::check_shape(shape, &d, false);
+  if (st != DFS_OK) return st;
+  if (!prm || !kv_idx || !kv_cnt || kcap < 1) return DFS_ERR_INVALID_ARG;
+  const long long rows = d.BH * d.nb;
+  if (rows > (1LL << 31) / 8) return DFS_ERR_UNSUPPORTED;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (prm->mode == DFS_SEL_LVSA) {
+    const long long P = (long long)d.H * d.W;
+    if (prm->lvsa_T_per < 1 || prm->lvsa_C < 1 || prm->lvsa_step < 0) return DFS_ERR_INVALID_ARG;
+    select_lvsa_kernel<<<grid, 256, 0, cs>>>((int)rows, d.nb, d.N, d.blk, (int)P, d.T, prm->lvsa_T_per,
+                                             prm->lvsa_C, prm->lvsa_step % prm->lvsa_T_per, kv_idx,
+                                             kv_cnt, kcap);
+    return dfs::launch_status();
+  }
+  if (!scores) return DFS_ERR_INVALID_ARG;
+  if (!dfs::aligned16(scores)) return DFS_ERR_MISALIGNED;
+  if (prm->mode == DFS_SEL_TOPK) {
+    if (prm->k < 0 || kcap < (prm->k < d.nb ? prm->k : d.nb)) return DFS_ERR_INVALID_ARG;
+  } else if (prm->mode == DFS_SEL_THRESHOLD) {
+    if (prm->cap < 0 || !(prm->tau >= 0.f) || kcap < (prm->cap < d.nb ? prm->cap : d.nb))
+      return DFS_ERR_INVALID_ARG;
+  } else {
+    return DFS_ERR_INVALID_ARG;
+  }
+  const int S = (d.nb + 31) / 32;
+#define DFS_SEL_LAUNCH(SS)                                                                       \
+  select_scores_kernel<SS><<<grid, 256, 0, cs>>>(scores, (int)rows, d.nb, prm->mode, prm->k,      \
+                                                 prm->cap, prm->tau, kv_idx, kv_cnt, kcap)
+  if (S <= 4) DFS_SEL_LAUNCH(4);
+  else if (S <= 8) DFS_SEL_LAUNCH(8);
+  else if (S <= 16) DFS_SEL_LAUNCH(16);
+  else if (S <= 32) DFS_SEL_LAUNCH(32);
+  else if (S <= 64) DFS_SEL_LAUNCH(64);
+  else return DFS_ERR_UNSUPPORTED;
+#undef DFS_SEL_LAUNCH
+  return dfs::launch_status();
+}

@@ -1,0 +1,183 @@
+"""Python binding of libdfsattn (argument marshalling only).
+
+Every function forwards to the C entry point of the same name declared in
+include/dfsattn.h; each stage of the path runs in the library's CUDA
+kernels. torch tensors supply device memory and the current CUDA stream.
+There is no fallback: if the library is missing or fails to load, importing
+this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdfsattn.so")
+
+DFS_OK = 0
+DFS_ERR_INVALID_ARG = -1
+DFS_ERR_UNSUPPORTED = -2
+DFS_ERR_MISALIGNED = -3
+DFS_ERR_CUDA = -4
+DFS_ERR_TIMEOUT = -5
+DFS_ERR_WORKSPACE = -6
+
+DFS_ORDER_RASTER = 0
+DFS_ORDER_HILBERT3D = 1
+DFS_SEL_TOPK = 0
+DFS_SEL_THRESHOLD = 1
+DFS_SEL_LVSA = 2
+DFS_WS_BLOCK_SCORE = 0
+
+DFS_FLAG_WAIT_TIMEOUT = 1
+DFS_FLAG_BAD_KV_INDEX = 2
+DFS_FLAG_KCAP_OVERFLOW = 4
+
+ORDERS = {"raster": DFS_ORDER_RASTER, "hilbert3d": DFS_ORDER_HILBERT3D}
+MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA}
+
+# C entry points declared in include/dfsattn.h.
+EXPORTS = (
+    "dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd", "dfs_unperm",
+    "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version",
+)
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "nh", "D", "T", "H", "W", "blk", "sb")]
+
+
+class _SelectParams(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("k", ctypes.c_int), ("cap", ctypes.c_int), ("tau", ctypes.c_float),
+                ("lvsa_T_per", ctypes.c_int), ("lvsa_C", ctypes.c_int), ("lvsa_step", ctypes.c_int)]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libdfsattn.so is not built ({_LIB_PATH}); run "
+                          "python -m block_sparse_attention_36_b200.build")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sp = ctypes.POINTER(_Shape)
+    lib.dfs_hilbert_perm.argtypes = [sp, I, P, P, I, P, P, P, P, P, P, P]
+    lib.dfs_block_score.argtypes = [sp, P, P, F, P, P, S, P]
+    lib.dfs_select_mask.argtypes = [sp, P, ctypes.POINTER(_SelectParams), P, P, I, P]
+    lib.dfs_sparse_attn_fwd.argtypes = [sp, P, P, P, P, P, I, F, P, P, P]
+    lib.dfs_unperm.argtypes = [sp, P, P, P, P]
+    lib.dfs_workspace_bytes.argtypes = [sp, I]
+    lib.dfs_workspace_bytes.restype = S
+    lib.dfs_get_error_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), I]
+    lib.dfs_status_string.argtypes = [I]
+    lib.dfs_status_string.restype = ctypes.c_char_p
+    lib.dfs_version.argtypes = []
+    for name in ("dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd",
+                 "dfs_unperm", "dfs_get_error_flags", "dfs_version"):
+        getattr(lib, name).restype = I
+    return lib
+
+
+LIB = _load()
+
+
+class DfsError(RuntimeError):
+    def __init__(self, call, status):
+        super().__init__(f"{call}: {LIB.dfs_status_string(status).decode()} ({status})")
+        self.status = status
+
+
+def _check(call, status):
+    if status != DFS_OK:
+        raise DfsError(call, status)
+
+
+@dataclass(frozen=True)
+class Shape:
+    B: int
+    nh: int
+    D: int
+    T: int
+    H: int
+    W: int
+    blk: int
+    sb: int
+
+    @property
+    def N(self):
+        return self.T * self.H * self.W
+
+    @property
+    def nb(self):
+        return -(-self.N // self.blk)
+
+    @property
+    def nsb(self):
+        return -(-self.N // self.sb)
+
+    def c(self):
+        return _Shape(self.B, self.nh, self.D, self.T, self.H, self.W, self.blk, self.sb)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dfs_hilbert_perm(shape: Shape, order, perm, inv, build_index, q, k, v, qp, kp, vp, stream=None):
+    order = ORDERS.get(order, order)
+    sh = shape.c()
+    _check("dfs_hilbert_perm", LIB.dfs_hilbert_perm(
+        ctypes.byref(sh), int(order), _ptr(perm), _ptr(inv), int(bool(build_index)),
+        _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp), _stream(stream)))
+
+
+def dfs_workspace_bytes(shape: Shape, which=DFS_WS_BLOCK_SCORE) -> int:
+    sh = shape.c()
+    return int(LIB.dfs_workspace_bytes(ctypes.byref(sh), int(which)))
+
+
+def dfs_block_score(shape: Shape, qp, kp, scale, scores, ws, stream=None):
+    sh = shape.c()
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("dfs_block_score", LIB.dfs_block_score(
+        ctypes.byref(sh), _ptr(qp), _ptr(kp), float(scale), _ptr(scores), _ptr(ws), nbytes, _stream(stream)))
+
+
+def select_params(mode, k=0, cap=0, tau=0.0, lvsa_T_per=8, lvsa_C=21, lvsa_step=0):
+    return _SelectParams(MODES.get(mode, mode), int(k), int(cap), float(tau), int(lvsa_T_per), int(lvsa_C),
+                         int(lvsa_step))
+
+
+def dfs_select_mask(shape: Shape, scores, params, kv_idx, kv_cnt, kcap, stream=None):
+    sh = shape.c()
+    _check("dfs_select_mask", LIB.dfs_select_mask(
+        ctypes.byref(sh), _ptr(scores), ctypes.byref(params), _ptr(kv_idx), _ptr(kv_cnt), int(kcap),
+        _stream(stream)))
+
+
+def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse=None, stream=None):
+    sh = shape.c()
+    _check("dfs_sparse_attn_fwd", LIB.dfs_sparse_attn_fwd(
+        ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
+        _ptr(op), _ptr(lse), _stream(stream)))
+
+
+def dfs_unperm(shape: Shape, perm, op, o, stream=None):
+    sh = shape.c()
+    _check("dfs_unperm", LIB.dfs_unperm(ctypes.byref(sh), _ptr(perm), _ptr(op), _ptr(o), _stream(stream)))
+
+
+def dfs_get_error_flags(clear=True) -> int:
+    v = ctypes.c_uint32(0)
+    _check("dfs_get_error_flags", LIB.dfs_get_error_flags(ctypes.byref(v), int(bool(clear))))
+    return int(v.value)
+
+
+def dfs_version() -> int:
+    return int(LIB.dfs_version())

@@ -1,0 +1,104 @@
+"""One DFSAttn attention layer on the GPU: buffers plus the five library calls.
+
+DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
+Generation, Methodology items 1-3: reorder tokens along the 3D Hilbert
+curve, score blocks hierarchically, select key blocks (the mask may be
+cached across denoising steps and refreshed at a fixed interval), attend
+over the kept blocks every step, restore the token order.
+
+This class only allocates device buffers (torch) and calls the C entry
+points in order; all arithmetic happens in libdfsattn's kernels.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import dfsattn as lib
+
+
+class DfsLayer:
+    def __init__(self, shape: lib.Shape, order="hilbert3d", mode="topk", k=0, cap=0, tau=0.0,
+                 lvsa_T_per=8, lvsa_C=21, lvsa_step=0, kcap=None, scale=0.0, device="cuda",
+                 want_lse=False):
+        self.shape = shape
+        self.order = order
+        self.mode = mode
+        self.params = lib.select_params(mode, k=k, cap=cap, tau=tau, lvsa_T_per=lvsa_T_per, lvsa_C=lvsa_C,
+                                        lvsa_step=lvsa_step)
+        s = shape
+        if kcap is None:
+            kcap = {"topk": max(1, min(k, s.nb)), "threshold": max(1, min(cap, s.nb))}.get(mode, s.nb)
+        self.kcap = int(kcap)
+        self.scale = float(scale) if scale and scale > 0 else 1.0 / math.sqrt(s.D)
+        dev = torch.device(device)
+        bf = torch.bfloat16
+        self.perm = torch.empty(s.N, dtype=torch.int32, device=dev)
+        self.inv = torch.empty(s.N, dtype=torch.int32, device=dev)
+        self.qp = torch.empty((s.B, s.nh, s.N, s.D), dtype=bf, device=dev)
+        self.kp = torch.empty_like(self.qp)
+        self.vp = torch.empty_like(self.qp)
+        self.op = torch.empty_like(self.qp)
+        self.out = torch.empty((s.B, s.N, s.nh, s.D), dtype=bf, device=dev)
+        self.lse = torch.empty((s.B, s.nh, s.N), dtype=torch.float32, device=dev) if want_lse else None
+        self.kv_idx = torch.full((s.B, s.nh, s.nb, self.kcap), -1, dtype=torch.int32, device=dev)
+        self.kv_cnt = torch.zeros((s.B, s.nh, s.nb), dtype=torch.int32, device=dev)
+        if mode != "lvsa":
+            self.scores = torch.empty((s.B, s.nh, s.nb, s.nb), dtype=torch.float32, device=dev)
+            nbytes = lib.dfs_workspace_bytes(s, lib.DFS_WS_BLOCK_SCORE)
+            self.ws = torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev)
+        else:
+            self.scores = None
+            self.ws = None
+        self._index_built = False
+
+    def set_budget(self, k=None, cap=None, tau=None, lvsa_step=None):
+        p = self.params
+        if k is not None:
+            if k > self.kcap and self.mode == "topk":
+                raise ValueError("k exceeds kcap")
+            p.k = int(k)
+        if cap is not None:
+            p.cap = int(cap)
+        if tau is not None:
+            p.tau = float(tau)
+        if lvsa_step is not None:
+            p.lvsa_step = int(lvsa_step)
+
+    def permute(self, q, k, v, stream=None):
+        lib.dfs_hilbert_perm(self.shape, self.order, self.perm, self.inv, not self._index_built, q, k, v,
+                             None if q is None else self.qp, None if k is None else self.kp,
+                             None if v is None else self.vp, stream)
+        self._index_built = True
+
+    def build_mask(self, stream=None):
+        if self.mode != "lvsa":
+            lib.dfs_block_score(self.shape, self.qp, self.kp, self.scale, self.scores, self.ws, stream)
+        lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
+
+    def attend(self, stream=None):
+        lib.dfs_sparse_attn_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt, self.kcap,
+                                self.scale, self.op, self.lse, stream)
+        lib.dfs_unperm(self.shape, self.perm, self.op, self.out, stream)
+
+    def forward(self, q, k, v, refresh_mask=True, stream=None):
+        """q, k, v: bf16 [B, N, nh, D] on the device (raster order). Returns the output buffer."""
+        self.permute(q, k, v, stream)
+        if refresh_mask:
+            self.build_mask(stream)
+        self.attend(stream)
+        return self.out
+
+    def kept_pairs(self):
+        """Valid (query, key) token pairs the kept blocks cover (for FLOP counts)."""
+        s = self.shape
+        rows_q = torch.full((s.nb,), s.blk, dtype=torch.int64)
+        rows_q[-1] = s.N - (s.nb - 1) * s.blk
+        idx = self.kv_idx.cpu().long()
+        cnt = self.kv_cnt.cpu().long()
+        pos = torch.arange(self.kcap).view(1, 1, 1, -1)
+        valid = pos < cnt.unsqueeze(-1)
+        keys = torch.where(idx == s.nb - 1, rows_q[-1], torch.full_like(idx, s.blk))
+        keys = torch.where(valid, keys, torch.zeros_like(keys)).sum(-1)   # [B, nh, nb]
+        return int((keys * rows_q.view(1, 1, -1)).sum())

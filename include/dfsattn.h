@@ -1,0 +1,183 @@
+/*
+ * libdfsattn -- the DFSAttn hot path on one B200 (sm_100a).
+ *
+ * Dynamic block-sparse spatiotemporal self-attention for video DiTs, as
+ * "DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
+ * Generation" describes it (Methodology items 1-3): reorder the T x H x W
+ * tokens along a global 3D Hilbert curve, score (query block, key block)
+ * pairs hierarchically from pooled sub-blocks, keep a budget of key blocks
+ * per query block, run block-sparse attention over the kept blocks only,
+ * and restore the token order. Two other selection rules share the path:
+ * the cumulative-mass threshold of "VMoBA: Mixture of Block Attention for
+ * Video Diffusion Models" (abstract, modification 3) and the frame mask of
+ * "LVSA: Training-Free Sparse Attention for Long Video Diffusion" (section 2).
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates or frees memory and keeps no state between
+ *     calls except a device-side error word (dfs_get_error_flags).
+ *   - Every tensor pointer must be 16-byte aligned; otherwise the call
+ *     returns DFS_ERR_MISALIGNED.
+ *   - Calls are asynchronous and ordered on `stream` (NULL = legacy default
+ *     stream). They never synchronise, print, abort or exit.
+ *   - The return value is a dfs_status. Argument errors are reported before
+ *     anything is launched; DFS_ERR_CUDA means a launch failed (the CUDA
+ *     error is left for cudaGetLastError to report).
+ *   - bf16 tensors use the IEEE-style bfloat16 layout (uint16 storage).
+ *   - Token order: "raster" index n = (t*H + h)*W + w; "curve" index i is the
+ *     position along the chosen order; perm[i] = n, inv[n] = i.
+ */
+#ifndef DFSATTN_H
+#define DFSATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st *dfs_stream_t;
+
+typedef enum {
+  DFS_OK = 0,
+  DFS_ERR_INVALID_ARG = -1, /* null pointer, bad size, inconsistent shape      */
+  DFS_ERR_UNSUPPORTED = -2, /* D, blk, blk/sb or nb outside the supported set  */
+  DFS_ERR_MISALIGNED = -3,  /* a tensor pointer is not 16-byte aligned          */
+  DFS_ERR_CUDA = -4,        /* a kernel launch or a CUDA runtime call failed    */
+  DFS_ERR_TIMEOUT = -5,     /* a bounded device wait gave up (see error flags)  */
+  DFS_ERR_WORKSPACE = -6    /* workspace missing or smaller than required       */
+} dfs_status;
+
+/* Problem shape.
+ *   B, nh, D : batch, heads, head dimension (D in {64, 128}).
+ *   T, H, W  : token grid; N = T*H*W tokens (N >= 1).
+ *   blk      : block size in tokens (64 or 128); nb = ceil(N / blk).
+ *   sb       : sub-block size in tokens; blk % sb == 0 and blk/sb in
+ *              {1, 2, 4, 8}; nsb = ceil(N / sb).                            */
+typedef struct {
+  int B, nh, D;
+  int T, H, W;
+  int blk, sb;
+} dfs_shape;
+
+enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1 };
+enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2 };
+enum { DFS_WS_BLOCK_SCORE = 0 };
+
+/* Device error word bits (dfs_get_error_flags). */
+enum {
+  DFS_FLAG_WAIT_TIMEOUT = 1u << 0, /* an mbarrier wait in the attention kernel gave up */
+  DFS_FLAG_BAD_KV_INDEX = 1u << 1, /* kv_idx held a block outside [0, nb): skipped     */
+  DFS_FLAG_KCAP_OVERFLOW = 1u << 2 /* a selected list was longer than kcap: truncated */
+};
+
+/* Selection settings for dfs_select_mask.
+ *   mode = DFS_SEL_TOPK      : keep the k highest-scoring key blocks of each
+ *                              row (equal scores: lower block index first).
+ *   mode = DFS_SEL_THRESHOLD : p = softmax over the row of the scores; keep
+ *                              the fewest best-ranked blocks whose mass
+ *                              reaches tau, at most cap of them.
+ *   mode = DFS_SEL_LVSA      : scores ignored (may be NULL). Query frame t
+ *                              attends to the anchors G_s = {f : (f - s) mod
+ *                              lvsa_T_per == 0} (s = lvsa_step) plus the
+ *                              (lvsa_C - |G_s|) nearest non-anchor frames
+ *                              (distance 0, 1, ..; t-d before t+d). Key block
+ *                              J is kept for query block I when a frame J
+ *                              touches lies in the union of the frame sets of
+ *                              the frames I touches. A frame is H*W tokens of
+ *                              the raster order.                              */
+typedef struct {
+  int mode;
+  int k;
+  int cap;
+  float tau;
+  int lvsa_T_per, lvsa_C, lvsa_step;
+} dfs_select_params;
+
+/* dfs_hilbert_perm -- token reorder (DFSAttn, Methodology item 1).
+ *
+ * If build_index != 0, first writes perm[N] and inv[N] (int32, device) for
+ * `order`: DFS_ORDER_HILBERT3D is the generalised 3D Hilbert curve over the
+ * whole T x H x W box (recursive box splitting; starts at (0,0,0), its major
+ * axis is the longest side, ties W, H, T); DFS_ORDER_RASTER is the identity.
+ * The index depends only on (T, H, W, order): callers build it once and
+ * reuse it with build_index = 0.
+ * Then gathers each non-NULL input x in {q, k, v}, bf16 [B, N, nh, D]
+ * (raster, token-major), into xp in {qp, kp, vp}, bf16 [B, nh, N, D]
+ * (curve order, head-major): xp[b, h, i, :] = x[b, perm[i], h, :].
+ * An input and its output must be both NULL or both non-NULL.             */
+int dfs_hilbert_perm(const dfs_shape *shape, int order, int32_t *perm, int32_t *inv,
+                     int build_index, const void *q, const void *k, const void *v,
+                     void *qp, void *kp, void *vp, dfs_stream_t stream);
+
+/* dfs_block_score -- hierarchical block scoring (DFSAttn, Methodology item 2).
+ *
+ * qp, kp: bf16 [B, nh, N, D] in curve order. Pools every run of sb tokens to
+ * its mean over the tokens that exist (fp32), then writes
+ *   scores[b, h, I, J] = scale * max_{i in I, j in J} qbar_i . kbar_j
+ * (fp32 [B, nh, nb, nb]; sub-blocks past N do not exist).
+ * scale <= 0 selects 1/sqrt(D).
+ * ws: device workspace of at least dfs_workspace_bytes(shape,
+ * DFS_WS_BLOCK_SCORE) bytes (the pooled means, fp32 [2, B, nh, nsb, D]);
+ * the call overwrites it, and it must stay untouched until the call's
+ * kernels finish.                                                          */
+int dfs_block_score(const dfs_shape *shape, const void *qp, const void *kp, float scale,
+                    float *scores, void *ws, size_t ws_bytes, dfs_stream_t stream);
+
+/* dfs_select_mask -- key-block selection (DFSAttn, Methodology item 3;
+ * VMoBA abstract, modification 3; LVSA section 2).
+ *
+ * scores: fp32 [B, nh, nb, nb] (NULL allowed for DFS_SEL_LVSA).
+ * Writes, per row (b, h, I), the kept key-block indices in ascending order
+ * to kv_idx[((b*nh + h)*nb + I)*kcap + 0 .. cnt-1] (int32) and cnt to
+ * kv_cnt[(b*nh + h)*nb + I]. Slots past cnt are not written. kcap >= 1; for
+ * top-k kcap >= min(k, nb) and for threshold kcap >= min(cap, nb) are
+ * checked on the host; a longer list is truncated to kcap and sets
+ * DFS_FLAG_KCAP_OVERFLOW.                                                  */
+int dfs_select_mask(const dfs_shape *shape, const float *scores, const dfs_select_params *params,
+                    int32_t *kv_idx, int32_t *kv_cnt, int kcap, dfs_stream_t stream);
+
+/* dfs_sparse_attn_fwd -- block-sparse attention over the kept blocks
+ * (DFSAttn, Methodology item 3 and Significance: block-wise execution).
+ *
+ * qp, kp, vp: bf16 [B, nh, N, D], curve order. For every query token q of
+ * query block I of head (b, h):
+ *   op[q] = sum_{k in kept(I), k < N} softmax_k(scale * q.k) v_k
+ * with kept(I) the tokens of the blocks kv_idx[row][0 .. kv_cnt[row]-1].
+ * A row with kv_cnt == 0 gets op = 0 (and lse = -inf).
+ * op: bf16 [B, nh, N, D]. lse (optional, fp32 [B, nh, N]): natural-log
+ * sum of exp of the scaled logits. scale <= 0 selects 1/sqrt(D).
+ * The softmax runs in fp32, P is rounded to bf16 for the P.V product,
+ * accumulation is fp32. Indices outside [0, nb) are skipped and set
+ * DFS_FLAG_BAD_KV_INDEX. Every device wait is bounded; a wait that gives up
+ * sets DFS_FLAG_WAIT_TIMEOUT and the kernel returns early.                */
+int dfs_sparse_attn_fwd(const dfs_shape *shape, const void *qp, const void *kp, const void *vp,
+                        const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
+                        void *op, float *lse, dfs_stream_t stream);
+
+/* dfs_unperm -- inverse reorder: o[b, perm[i], h, :] = op[b, h, i, :],
+ * op bf16 [B, nh, N, D] (curve order) -> o bf16 [B, N, nh, D] (raster).   */
+int dfs_unperm(const dfs_shape *shape, const int32_t *perm, const void *op, void *o,
+               dfs_stream_t stream);
+
+/* Workspace bytes a call needs (0 if none). which: DFS_WS_*. Returns 0 for
+ * an invalid shape.                                                        */
+size_t dfs_workspace_bytes(const dfs_shape *shape, int which);
+
+/* Reads the device error word of the current device (DFS_FLAG_* bits) into
+ * *flags; clears it when clear != 0. Synchronises the current device.     */
+int dfs_get_error_flags(uint32_t *flags, int clear);
+
+/* Static text for a dfs_status value. */
+const char *dfs_status_string(int status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int dfs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFSATTN_H */

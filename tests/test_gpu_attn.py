@@ -1,0 +1,141 @@
+"""GPU block-sparse attention against the fp64 oracle.
+
+Page: DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
+Generation, Methodology item 3 and Significance (block-wise execution over
+the kept blocks). Tolerance: max abs <= 2e-2, relative Frobenius <= 5e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention
+from tests.parity import assert_attn_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib(cuda_device):
+    from block_sparse_attention_36_b200 import dfsattn
+    return dfsattn
+
+
+def _lists(rng, B, nh, nb, kcap, full=False):
+    idx = np.full((B, nh, nb, kcap), -1, dtype=np.int32)
+    cnt = np.zeros((B, nh, nb), dtype=np.int32)
+    for b in range(B):
+        for h in range(nh):
+            for I in range(nb):
+                c = nb if full else int(rng.integers(0, min(kcap, nb) + 1))
+                c = min(c, kcap)
+                js = np.sort(rng.choice(nb, size=c, replace=False)) if c else np.zeros(0, np.int32)
+                idx[b, h, I, :c] = js
+                cnt[b, h, I] = c
+    return idx, cnt
+
+
+def _run(lib, q, k, v, idx, cnt, D, blk, N, scale=0.0, want_lse=True):
+    B, nh = q.shape[0], q.shape[1]
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, 16)
+    op = torch.empty((B, nh, N, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, nh, N), dtype=torch.float32, device="cuda") if want_lse else None
+    lib.dfs_sparse_attn_fwd(s, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(idx).cuda(),
+                            torch.from_numpy(cnt).cuda(), idx.shape[-1], scale, op, lse)
+    torch.cuda.synchronize()
+    return op.float().cpu().numpy(), (lse.cpu().numpy() if want_lse else None)
+
+
+CASES = [  # B, nh, D, blk, N
+    (1, 2, 128, 128, 1000),    # ragged last block (104)
+    (1, 2, 128, 128, 4096),
+    (2, 1, 64, 64, 2048),      # tiny workload geometry
+    (1, 2, 64, 64, 1000),      # ragged (40)
+    (1, 1, 128, 64, 700),
+    (1, 1, 64, 128, 700),
+]
+
+
+@pytest.mark.parametrize("B,nh,D,blk,N", CASES)
+def test_random_lists(lib, B, nh, D, blk, N):
+    rng = np.random.default_rng(N + D)
+    g = torch.Generator().manual_seed(N)
+    q = torch.randn((B, nh, N, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, nh, N, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, nh, N, D), generator=g).to(torch.bfloat16)
+    nb = -(-N // blk)
+    kcap = max(1, nb // 2 + 1)
+    idx, cnt = _lists(rng, B, nh, nb, kcap)
+    got, lse = _run(lib, q, k, v, idx, cnt, D, blk, N)
+    ref, rlse = attention.block_sparse_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                                 idx, cnt, blk)
+    assert_attn_close(got, ref, "output")
+    fin = np.isfinite(rlse)
+    assert np.array_equal(fin, np.isfinite(lse))
+    assert np.abs(lse[fin] - rlse[fin]).max() < 1e-3
+
+
+@pytest.mark.parametrize("D,blk", [(128, 128), (64, 64)])
+def test_full_mask_is_dense(lib, D, blk):
+    N = 640 if blk == 128 else 576
+    g = torch.Generator().manual_seed(7)
+    q, k, v = (torch.randn((1, 2, N, D), generator=g).to(torch.bfloat16) for _ in range(3))
+    nb = -(-N // blk)
+    idx, cnt = _lists(np.random.default_rng(0), 1, 2, nb, nb, full=True)
+    got, _ = _run(lib, q, k, v, idx, cnt, D, blk, N)
+    ref = attention.dense_attention(q.double().numpy(), k.double().numpy(), v.double().numpy())
+    assert_attn_close(got, ref, "dense")
+
+
+def test_peaked_logits_and_rescale(lib):
+    # Large logits make the running maximum jump between blocks, which
+    # exercises the O rescale path; scale is passed explicitly.
+    N, D, blk = 1024, 128, 128
+    g = torch.Generator().manual_seed(11)
+    q = (torch.randn((1, 1, N, D), generator=g) * 3).to(torch.bfloat16)
+    k = (torch.randn((1, 1, N, D), generator=g) * 3).to(torch.bfloat16)
+    k[:, :, 700:710] *= 4
+    v = torch.randn((1, 1, N, D), generator=g).to(torch.bfloat16)
+    nb = N // blk
+    idx, cnt = _lists(np.random.default_rng(1), 1, 1, nb, nb, full=True)
+    got, _ = _run(lib, q, k, v, idx, cnt, D, blk, N, scale=0.2)
+    ref, _ = attention.block_sparse_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                              idx, cnt, blk, 0.2)
+    assert_attn_close(got, ref, "peaked")
+
+
+def test_empty_rows_and_bad_indices(lib):
+    N, D, blk = 512, 64, 64
+    g = torch.Generator().manual_seed(5)
+    q, k, v = (torch.randn((1, 1, N, D), generator=g).to(torch.bfloat16) for _ in range(3))
+    nb = N // blk
+    idx = np.full((1, 1, nb, 4), -1, dtype=np.int32)
+    cnt = np.zeros((1, 1, nb), dtype=np.int32)
+    idx[0, 0, 1, :3] = [0, 99, 5]          # 99 is out of range: skipped, flagged
+    cnt[0, 0, 1] = 3
+    idx[0, 0, 2, :2] = [2, 3]
+    cnt[0, 0, 2] = 2
+    lib.dfs_get_error_flags(clear=True)
+    got, lse = _run(lib, q, k, v, idx, cnt, D, blk, N)
+    assert lib.dfs_get_error_flags(clear=True) & lib.DFS_FLAG_BAD_KV_INDEX
+    clean_idx, clean_cnt = idx.copy(), cnt.copy()
+    clean_idx[0, 0, 1, :3] = [0, 5, -1]
+    clean_cnt[0, 0, 1] = 2
+    ref, rlse = attention.block_sparse_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                                 clean_idx, clean_cnt, blk)
+    assert_attn_close(got, ref, "bad indices")
+    assert (got[0, 0, :64] == 0).all() and np.isneginf(lse[0, 0, :64]).all()
+
+
+def test_constant_v(lib):
+    N, D, blk = 384, 128, 128
+    g = torch.Generator().manual_seed(2)
+    q, k = (torch.randn((1, 1, N, D), generator=g).to(torch.bfloat16) for _ in range(2))
+    v = torch.full((1, 1, N, D), 0.75).to(torch.bfloat16)
+    nb = N // blk
+    idx, cnt = _lists(np.random.default_rng(3), 1, 1, nb, 2)
+    cnt[cnt == 0] = 1
+    idx[..., 0] = np.where(idx[..., 0] < 0, 0, idx[..., 0])
+    got, _ = _run(lib, q, k, v, idx, cnt, D, blk, N)
+    assert np.abs(got - 0.75).max() < 4e-3

@@ -1,0 +1,69 @@
+"""GPU pooling and hierarchical block scores against the fp64 oracle.
+
+Page: DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
+Generation, Methodology item 2. The GPU computes in fp32; the bound used
+here is the fp32 rounding of sums of <= sb bf16 values and of D-term dot
+products (relative error ~ (D + sb) * 2^-24 of the magnitudes summed)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import scoring
+
+pytestmark = pytest.mark.gpu
+
+U32 = 2.0 ** -24
+
+
+@pytest.fixture(scope="module")
+def lib(cuda_device):
+    from block_sparse_attention_36_b200 import dfsattn
+    return dfsattn
+
+
+def _run(lib, B, nh, D, N, blk, sb, seed=0, scale=0.0):
+    g = torch.Generator().manual_seed(seed)
+    qp = torch.randn((B, nh, N, D), generator=g).to(torch.bfloat16)
+    kp = (torch.randn((B, nh, N, D), generator=g) + 0.3).to(torch.bfloat16)
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, sb)
+    scores = torch.empty((B, nh, s.nb, s.nb), dtype=torch.float32, device="cuda")
+    ws = torch.empty(lib.dfs_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    lib.dfs_block_score(s, qp.cuda(), kp.cuda(), scale, scores, ws)
+    torch.cuda.synchronize()
+    pooled = ws.view(torch.float32).view(2, B, nh, s.nsb, D).cpu().numpy()
+    return qp, kp, scores.cpu().numpy(), pooled, s
+
+
+CASES = [
+    (1, 2, 64, 2048, 64, 16),     # tiny workload
+    (1, 3, 128, 1000, 128, 32),   # ragged: last block 104 tokens, last sub-block 8
+    (2, 2, 128, 777, 128, 16),    # r = 8
+    (1, 2, 64, 300, 64, 32),      # r = 2
+    (1, 1, 128, 513, 128, 128),   # r = 1 (coarse block pooling)
+    (1, 2, 128, 32760, 128, 32),  # full Wan-layer sequence, two heads
+]
+
+
+@pytest.mark.parametrize("B,nh,D,N,blk,sb", CASES)
+def test_pool_and_scores(lib, B, nh, D, N, blk, sb):
+    qp, kp, got, pooled, s = _run(lib, B, nh, D, N, blk, sb)
+    q64, k64 = qp.double().numpy(), kp.double().numpy()
+    oq, ok = scoring.pool_subblocks(q64, sb), scoring.pool_subblocks(k64, sb)
+    tol_pool = (sb + 2) * U32 * max(np.abs(q64).max(), np.abs(k64).max())
+    assert np.abs(pooled[0] - oq).max() <= tol_pool
+    assert np.abs(pooled[1] - ok).max() <= tol_pool
+    scale = 1.0 / math.sqrt(D)
+    ref = scoring.block_scores(q64, k64, blk, sb, scale)
+    # per-entry bound: (D + 2 sb + 4) u * scale * max |qbar| |kbar| summed over d
+    mag = scale * D * np.abs(oq).max() * np.abs(ok).max()
+    tol = (D + 2 * sb + 4) * U32 * mag
+    err = np.abs(got - ref).max()
+    assert err <= tol, (err, tol)
+
+
+def test_explicit_scale(lib):
+    qp, kp, got, _, s = _run(lib, 1, 1, 64, 500, 64, 16, seed=3, scale=0.5)
+    ref = scoring.block_scores(qp.double().numpy(), kp.double().numpy(), 64, 16, 0.5)
+    assert np.abs(got - ref).max() < 1e-4
