@@ -5,30 +5,45 @@
 // attention runs block-wise over the kept blocks only, on the reordered,
 // contiguous token blocks.
 //
-// One CTA computes one 128-row query tile (one query block; for 64-token
-// blocks the lower 64 rows) of one head against the key blocks of its list.
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q once, then K and V tiles of each kept block
-//              into a 2-stage ring (128-byte swizzled tiles, no multicast).
-//   warp 1     owns tensor memory; one lane issues the tcgen05 MMAs:
-//                S_j = Q K_j^T  (SS, into TMEM buffer j % 2)
-//                O  += P_j V_j  (TS: P_j read back from TMEM, V_j MN-major)
-//              issuing S_{j+1} before waiting for P_j, so the tensor pipe
-//              works on the next logits while the softmax runs.
-//   warps 2-5  softmax, one thread per query row: fp32 online softmax on S
-//              read from TMEM, P_j written back into S_j's columns as bf16;
-//              O is rescaled in TMEM only when the running row maximum grows
-//              by more than 2^8 (an older maximum is exact as long as the
-//              same one is used for P and for the row sum); epilogue
-//              normalises O and writes bf16 rows (and the log-sum-exp).
-// Tensor memory: S0 | S1 | O  (BLK + BLK + D fp32 columns, 128 lanes).
-// Every mbarrier wait is bounded (DFS_FLAG_WAIT_TIMEOUT, early return).
+// A CTA owns two query tiles ("slots" A and B: query blocks 2x and 2x+1 of
+// one head), each with its own kept list. While the softmax of one slot
+// runs, the tensor pipe works on the other slot's products, so neither the
+// tensor pipe nor the exponential units wait on each other for long.
+// Warp roles (384 threads, three warpgroups):
+//   warp 0     TMA producer: Q_A, Q_B, then the K and V tiles of both lists
+//              into a 4-stage ring, in exactly the order the MMAs consume
+//              them (128-byte swizzled tiles, no multicast).
+//   warp 1     owns tensor memory; one lane issues the tcgen05 MMAs, per
+//              slot X and kept block j:
+//                S_X = Q_X K_j^T  (SS)            into TMEM S_X
+//                O_X += P_X V_j   (TS: P_X from TMEM, V MN-major)
+//              ordered S_A(0) S_B(0), then per j: PV_A(j) S_A(j+1)
+//              PV_B(j) S_B(j+1); S_X(j+1) overwrites P_X(j) only after
+//              PV_X(j) read it (tcgen05 MMAs of one thread run in order).
+//   warps 2-3  compact the two kept lists into shared memory, then idle.
+//   warps 4-7  softmax of slot A, warps 8-11 softmax of slot B: one thread
+//              per query row; fp32 online softmax on S read from TMEM,
+//              P written back as bf16 over S_X; O_X is rescaled in TMEM
+//              only when a warp's running maximum grows by more than 2^8
+//              (an older maximum stays exact as long as P and the row sum
+//              use the same one); epilogue normalises O_X and stores bf16
+//              rows and the log-sum-exp.
+// Tensor memory: S_A | S_B | O_A | O_B (BLK, BLK, D, D fp32 columns).
+// Every mbarrier wait is bounded (DFS_FLAG_WAIT_TIMEOUT, early return);
+// copies and MMAs in flight are drained before tensor memory is released.
 #include <cuda.h>
 
 #include <mutex>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
+
+// Every DFS_ATTN_EXP2_EMU-th pair of softmax exponentials is computed on the
+// FMA pipe (0: all on the special-function unit).
+#ifndef DFS_ATTN_EXP2_EMU
+#define DFS_ATTN_EXP2_EMU 0
+#endif
 
 namespace {
 
@@ -36,37 +51,61 @@ using namespace dfs::sm100;
 
 __device__ uint32_t g_attn_flags;
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per pipeline wait
-constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s per drain wait
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
-constexpr int kQRows = 128;  // MMA M
+// Wait limits in SM clock cycles (about 2 s and 1 s at the 2 GHz maximum).
+constexpr long long kWaitLimit = 4000000000ll;   // per pipeline wait
+constexpr long long kDrainLimit = 2000000000ll;  // per drain wait
+constexpr int kRing = 4;                           // K/V ring stages
+constexpr int kThreads = 384;                      // 3 warpgroups
+constexpr int kQRows = 128;                        // MMA M
 
 template <int D, int BLK>
 struct Cfg {
-  static constexpr int kChunks = D / 64;                   // 128-byte column slabs per row
-  static constexpr int kQBytes = kQRows * D * 2;
-  static constexpr int kKVBytes = BLK * D * 2;
+  static constexpr int kChunks = D / 64;          // 128-byte column slabs per row
+  static constexpr int kQBytes = kQRows * D * 2;  // one slot's Q tile
+  static constexpr int kTileBytes = BLK * D * 2;  // one K or V tile
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kVOff = kKOff + kStages * kKVBytes;
-  static constexpr int kBarOff = kVOff + kStages * kKVBytes;
-  static constexpr int kTmemCols = (2 * BLK + D <= 256) ? 256 : 512;
-  static constexpr int kS0 = 0, kS1 = BLK, kO = 2 * BLK;
+  static constexpr int kRingOff = 2 * kQBytes;
+  static constexpr int kBarOff = kRingOff + kRing * kTileBytes;
+  static constexpr int kCols = 2 * BLK + 2 * D;
+  static constexpr int kTmemCols = kCols <= 256 ? 256 : 512;
+  __host__ __device__ static constexpr int s_col(int x) { return x * BLK; }
+  __host__ __device__ static constexpr int o_col(int x) { return 2 * BLK + x * D; }
 };
 
 struct __align__(8) Barriers {
-  uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_ready, o_final;
+  uint64_t q_full[2];
+  uint64_t kv_full[kRing], kv_empty[kRing];
+  uint64_t s_full[2], p_full[2], o_final[2];
+  uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
-  int n_kv;
+  int n_kv[2];
 };
 
+// S = Q K^T for one 128-row query tile and one key tile: D/16 MMAs of
+// K = 16; dq, dk describe the first 16 columns of the 128-byte-swizzled tiles.
 template <int D, int BLK>
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t dk) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kQRows, BLK, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t oa = (uint64_t)(((kk >> 2) * (kQRows * 128) + (kk & 3) * 32) >> 4);
+    const uint64_t ob = (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
+    mma_ss(d_tmem, dq + oa, dk + ob, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V for one query tile: P (bf16) from tensor memory, V MN-major in
+// shared memory; BLK/16 MMAs of K = 16.
+template <int D, int BLK>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kQRows, D, 1);
+#pragma unroll
+  for (int kk = 0; kk < BLK / 16; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int D, int BLK, int EMU>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ kv_idx,
@@ -74,182 +113,206 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 __nv_bfloat16* __restrict__ op, float* __restrict__ lse, int max_list) {
   using C = Cfg<D, BLK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte alignment for the 128-byte-swizzled tiles.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kBarOff);
-  int32_t* list = reinterpret_cast<int32_t*>(smem + C::kBarOff + sizeof(Barriers));
+  int32_t* lists = reinterpret_cast<int32_t*>(smem + C::kBarOff + sizeof(Barriers));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int I = blockIdx.x;
   const int bh = blockIdx.y;
-  const long long row_id = (long long)bh * nb + I;
+  const int I0 = 2 * blockIdx.x;  // slot A: I0, slot B: I0 + 1
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
-      mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->q_full[x], 1);
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_full[x], 4);
+      mbar_init(&bars->o_final[x], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], 4);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->o_ready, 1);
-    mbar_init(&bars->o_final, 1);
+    mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
-    // Compact the kept list into shared memory, dropping invalid indices.
-    int cnt = kv_cnt[row_id];
-    cnt = max(0, min(cnt, min(kcap, max_list)));
-    const int32_t* src = kv_idx + row_id * (long long)kcap;
+  if (warp == 2 || warp == 3) {
+    // Compact the slot's kept list into shared memory, dropping invalid indices.
+    const int x = warp - 2;
+    const int I = I0 + x;
     int base = 0;
     bool bad = false;
-    for (int j0 = 0; j0 < cnt; j0 += 32) {
-      const int j = j0 + lane;
-      int J = -1;
-      if (j < cnt) J = src[j];
-      const bool ok = (j < cnt) && J >= 0 && J < nb;
-      bad |= (j < cnt) && !ok;
-      const unsigned m = __ballot_sync(0xffffffffu, ok);
-      if (ok) list[base + __popc(m & ((1u << lane) - 1u))] = J;
-      base += __popc(m);
+    if (I < nb) {
+      const long long row_id = (long long)bh * nb + I;
+      int cnt = kv_cnt[row_id];
+      cnt = max(0, min(cnt, min(kcap, max_list)));
+      const int32_t* src = kv_idx + row_id * (long long)kcap;
+      int32_t* dst = lists + x * max_list;
+      for (int j0 = 0; j0 < cnt; j0 += 32) {
+        const int j = j0 + lane;
+        int J = -1;
+        if (j < cnt) J = src[j];
+        const bool ok = (j < cnt) && J >= 0 && J < nb;
+        bad |= (j < cnt) && !ok;
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        if (ok) dst[base + __popc(m & ((1u << lane) - 1u))] = J;
+        base += __popc(m);
+      }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_attn_flags, (uint32_t)DFS_FLAG_BAD_KV_INDEX);
-    if (lane == 0) bars->n_kv = base;
+    if (lane == 0) bars->n_kv[x] = base;
   }
   if (warp == 1) tmem_alloc(&bars->tmem_base, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const int n_kv = bars->n_kv;
-
+  const int n[2] = {bars->n_kv[0], bars->n_kv[1]};
+  const int jmax = max(n[0], n[1]);
+  if (warp < 4) {
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensor_map(&tm_q);
       prefetch_tensor_map(&tm_k);
       prefetch_tensor_map(&tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, C::kQBytes);
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(smem + C::kQOff + c * (kQRows * 128), &tm_q, &bars->q_full, c * 64, I * BLK, bh);
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % kStages;
-        const uint32_t ph = (uint32_t)((j / kStages) & 1);
-        const int J = list[j];
-        if (!mbar_wait_bounded(&bars->k_empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) break;
-        mbar_arrive_expect_tx(&bars->k_full[s], C::kKVBytes);
+      for (int x = 0; x < 2; ++x) {
+        if (n[x] == 0) continue;
+        mbar_arrive_expect_tx(&bars->q_full[x], C::kQBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(smem + C::kKOff + s * C::kKVBytes + c * (BLK * 128), &tm_k, &bars->k_full[s], c * 64,
-                      J * BLK, bh);
-        issued_k = j + 1;
-        if (!mbar_wait_bounded(&bars->v_empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) break;
-        mbar_arrive_expect_tx(&bars->v_full[s], C::kKVBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(smem + C::kVOff + s * C::kKVBytes + c * (BLK * 128), &tm_v, &bars->v_full[s], c * 64,
-                      J * BLK, bh);
-        issued_v = j + 1;
+          tma_load_3d(smem + C::kQOff + x * C::kQBytes + c * (kQRows * 128), &tm_q, &bars->q_full[x], c * 64,
+                      (I0 + x) * BLK, bh);
       }
-      // Drain: every load issued must land before the CTA may exit. A stage
-      // is reloaded only after its previous load was consumed, so only the
-      // last kStages loads of each ring can still be in flight.
-      for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
-        mbar_wait_timed(&bars->k_full[j % kStages], (uint32_t)((j / kStages) & 1), kDrainLimitNs);
-      for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
-        mbar_wait_timed(&bars->v_full[j % kStages], (uint32_t)((j / kStages) & 1), kDrainLimitNs);
-      mbar_wait_timed(&bars->q_full, 0, kDrainLimitNs);
+      // Same step order as the MMA issuer: step -1 loads K_A(0), K_B(0); step
+      // j loads, per slot, V(j) and then K(j+1).
+      int t = 0;  // ring tiles loaded so far
+      bool ok = true;
+      for (int step = -1; step < jmax && ok; ++step) {
+#pragma unroll 1
+        for (int x = 0; x < 2; ++x) {
+          const int nx = n[x];
+          if (step >= nx) continue;
+#pragma unroll 1
+          for (int kind = 0; kind < 2; ++kind) {      // 0: V(step), 1: K(step + 1)
+            const int jj = kind == 0 ? step : step + 1;
+            if (jj < 0 || jj >= nx) continue;
+            const int st = t % kRing;
+            if (!mbar_wait_bounded(&bars->kv_empty[st], (uint32_t)(((t / kRing) & 1) ^ 1), abort_flag, kWaitLimit)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bars->kv_full[st], C::kTileBytes);
+            const int J = lists[x * max_list + jj];
+            uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
+            const CUtensorMap* map = kind == 0 ? &tm_v : &tm_k;
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(dst + c * (BLK * 128), map, &bars->kv_full[st], c * 64, J * BLK, bh);
+            ++t;
+          }
+          if (!ok) break;
+        }
+      }
+      // Drain: a stage is reloaded only after its previous tile was
+      // consumed, so only the last kRing loads can still be in flight.
+      for (int u = max(0, t - kRing); u < t; ++u)
+        mbar_wait_timed(&bars->kv_full[u % kRing], (uint32_t)((u / kRing) & 1), kDrainLimit);
+      for (int x = 0; x < 2; ++x)
+        if (n[x] > 0) mbar_wait_timed(&bars->q_full[x], 0, kDrainLimit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kQRows, BLK, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kQRows, D, 1);
-      const uint32_t q_base = smem_addr(smem + C::kQOff);
-      const uint32_t k_base = smem_addr(smem + C::kKOff);
-      const uint32_t v_base = smem_addr(smem + C::kVOff);
-      bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimitNs);
-      auto issue_pv = [&](int jj) -> bool {
-        const int b = jj & 1, s = jj % kStages;
-        const uint32_t ph = (uint32_t)((jj / kStages) & 1);
-        if (!mbar_wait_bounded(&bars->p_full[b], (uint32_t)((jj >> 1) & 1), abort_flag, kWaitLimitNs)) return false;
-        if (!mbar_wait_bounded(&bars->v_full[s], ph, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + (b ? C::kS1 : C::kS0);
-        const uint32_t vs = v_base + s * C::kKVBytes;
-#pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
-          const uint64_t bdesc = desc_sw128(vs + kk * 2048, BLK * 128, 1024);
-          mma_ts(tmem + C::kO, p_tmem + kk * 8, bdesc, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+      // Descriptors are built once; a K step or a ring stage only moves the
+      // start-address field (16-byte units), so each MMA costs an add.
+      const uint64_t dq = desc_sw128(smem_addr(smem + C::kQOff), 16, 1024);
+      const uint64_t dk = desc_sw128(smem_addr(smem + C::kRingOff), 16, 1024);
+      const uint64_t dv = desc_sw128(smem_addr(smem + C::kRingOff), BLK * 128, 1024);
+      bool ok = true;
+      for (int x = 0; x < 2 && ok; ++x)
+        if (n[x] > 0) ok = mbar_wait_bounded(&bars->q_full[x], 0, abort_flag, kWaitLimit);
+      // Step -1 issues S_A(0), S_B(0); step j issues, per slot, PV(j) and
+      // then S(j+1) (or the slot's final commit).
+      int t = 0;  // ring tiles consumed so far
+      for (int step = -1; step < jmax && ok; ++step) {
+#pragma unroll 1
+        for (int x = 0; x < 2; ++x) {
+          const int nx = n[x];
+          if (step >= nx) continue;
+          if (step >= 0) {
+            // P_X was written by other threads with tcgen05.st: order this
+            // thread's MMAs after their arrival. (TMA-filled tiles need no
+            // fence: the mbarrier transaction count orders them.)
+            if (!mbar_wait_bounded(&bars->p_full[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+            tc_fence_after();
+            const int st = t % kRing;
+            if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+            issue_pv<D, BLK>(tmem + C::o_col(x), tmem + C::s_col(x), dv + (uint64_t)((st * C::kTileBytes) >> 4),
+                             step > 0);
+            mma_commit(&bars->kv_empty[st]);
+            ++t;
+          }
+          if (step + 1 < nx) {
+            const int st = t % kRing;
+            if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+            issue_s<D, BLK>(tmem + C::s_col(x), dq + (uint64_t)((x * C::kQBytes) >> 4),
+                            dk + (uint64_t)((st * C::kTileBytes) >> 4));
+            mma_commit(&bars->s_full[x]);
+            mma_commit(&bars->kv_empty[st]);
+            ++t;
+          } else if (step >= 0) {
+            mma_commit(&bars->o_final[x]);
+          }
         }
-        mma_commit(&bars->v_empty[s]);
-        mma_commit(&bars->o_ready);
-        return true;
-      };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % kStages, b = j & 1;
-        const uint32_t ph = (uint32_t)((j / kStages) & 1);
-        if (!mbar_wait_bounded(&bars->k_full[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t ks = k_base + s * C::kKVBytes;
-        const uint32_t s_tmem = tmem + (b ? C::kS1 : C::kS0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int c = kk >> 2, w = kk & 3;
-          const uint64_t adesc = desc_sw128(q_base + c * (kQRows * 128) + w * 32, 16, 1024);
-          const uint64_t bdesc = desc_sw128(ks + c * (BLK * 128) + w * 32, 16, 1024);
-          mma_ss(s_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->s_full[b]);
-        mma_commit(&bars->k_empty[s]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
-      if (ok && n_kv > 0) issue_pv(n_kv - 1);
-      mma_commit(&bars->o_final);
-      // Every MMA of this CTA must finish before tensor memory is released.
-      mbar_wait_timed(&bars->o_final, 0, kDrainLimitNs);
+      // Every MMA must finish before tensor memory is released.
+      mma_commit(&bars->mma_done);
+      mbar_wait_timed(&bars->mma_done, 0, kDrainLimit);
     }
     __syncwarp();
+  }
   } else {
     // ------------------------------------------------------------ softmax
-    const int sub = warp & 3;                        // TMEM lane quarter of this warp
-    const int r = sub * 32 + lane;                   // query row in the tile
+    const int x = warp < 8 ? 0 : 1;                 // slot
+    const int I = I0 + x;
+    const int sub = warp & 3;                       // TMEM lane quarter of this warp
+    const int r = sub * 32 + lane;                  // query row in the tile
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-    const int rem = N - (nb - 1) * BLK;              // valid keys in the last block
-    float m = -INFINITY;                             // running max (log2 units)
-    float l = 0.f;                                   // running row sum
+    const uint32_t s_addr = tmem + lane_base + C::s_col(x);
+    const uint32_t o_addr = tmem + lane_base + C::o_col(x);
+    const int rem = N - (nb - 1) * BLK;             // valid keys in the last block
+    const int32_t* list = lists + x * max_list;
+    const int nx = n[x];
+    float m = -INFINITY;                            // running max (log2 units)
+    float l = 0.f;                                  // running row sum
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait_bounded(&bars->s_full[b], (uint32_t)((j >> 1) & 1), abort_flag, kWaitLimitNs)) { ok = false; break; }
+    for (int j = 0; j < nx; ++j) {
+      if (!mbar_wait_bounded(&bars->s_full[x], (uint32_t)(j & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + (b ? C::kS1 : C::kS0);
       float sv[BLK];
 #pragma unroll
       for (int c = 0; c < BLK / 32; ++c) {
         uint32_t raw[32];
         tmem_ld32(s_addr + c * 32, raw);
-        tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[e]);
       }
-      const int J = list[j];
-      if (J == nb - 1 && rem < BLK) {
+      tmem_wait_ld();
+      if (list[j] == nb - 1 && rem < BLK) {
 #pragma unroll
         for (int e = 0; e < BLK; ++e)
           if (e >= rem) sv[e] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row maximum, eight independent chains
+      float mx8[8];
 #pragma unroll
-      for (int e = 0; e < BLK; ++e) mx = fmaxf(mx, sv[e]);
+      for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+#pragma unroll
+      for (int e = 8; e < BLK; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], sv[e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_blk = mx * scale_log2;
-      // Keep the old maximum unless it is more than 2^8 below the new one
-      // somewhere in this warp; then the warp rescales O and its sums.
       bool rescale = false;
       float m_use;
       if (j == 0) {
@@ -258,36 +321,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         rescale = __any_sync(0xffffffffu, m_blk > m + 8.0f);
         m_use = rescale ? fmaxf(m, m_blk) : m;
       }
-      // P = exp2(s * scale_log2 - m), bf16, written over S_j's first columns
-      // (S_j is fully read already; PV_{j-1} reads the other buffer).
-      float rs = 0.f;
+      // P = 2^(s * scale_log2 - m), bf16, written over S_X (fully read).
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 acc[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < BLK / 64; ++c) {
         uint32_t packed[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2(fmaf(sv[c * 64 + 2 * e], scale_log2, -m_use));
-          const float p1 = ex2(fmaf(sv[c * 64 + 2 * e + 1], scale_log2, -m_use));
-          rs += p0 + p1;
-          packed[e] = pack_bf16x2(p0, p1);
+          const float2 x2 = __ffma2_rn(make_float2(sv[c * 64 + 2 * e], sv[c * 64 + 2 * e + 1]), sc2, nm2);
+          float2 p2;
+          if (EMU > 0 && (e % (EMU > 0 ? EMU : 1)) == EMU - 1) {
+            p2 = make_float2(dfs::exp2_poly(x2.x), dfs::exp2_poly(x2.y));
+          } else {
+            p2 = make_float2(ex2(x2.x), ex2(x2.y));
+          }
+          acc[e & 3] = __fadd2_rn(acc[e & 3], p2);
+          packed[e] = pack_bf16x2(p2.x, p2.y);
         }
         tmem_st32(s_addr + c * 32, packed);
       }
-      // One o_ready phase per iteration: PV_{j-1} has finished with O.
-      if (j >= 1) {
-        if (!mbar_wait_bounded(&bars->o_ready, (uint32_t)((j - 1) & 1), abort_flag, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-      }
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a = __fadd2_rn(a01, a23);
+      const float rs = a.x + a.y;
+      // O_X may be rescaled here: s_full(j) was committed after PV_X(j-1)
+      // by the same thread, so PV_X(j-1) has completed.
       if (rescale) {
         const float alpha = ex2(m - m_use);
-        const uint32_t o_addr = tmem + lane_base + C::kO;
+        const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t raw[32];
           tmem_ld32(o_addr + c * 32, raw);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+          for (int e = 0; e < 16; ++e) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(raw[2 * e]), __uint_as_float(raw[2 * e + 1])), al2);
+            raw[2 * e] = __float_as_uint(v.x);
+            raw[2 * e + 1] = __float_as_uint(v.y);
+          }
           tmem_st32(o_addr + c * 32, raw);
         }
         l *= alpha;
@@ -297,20 +372,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       l += rs;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[b]);
+      if (lane == 0) mbar_arrive(&bars->p_full[x]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = mbar_wait_bounded(&bars->o_final, 0, abort_flag, kWaitLimitNs);
+    if (ok && nx > 0) ok = mbar_wait_bounded(&bars->o_final[x], 0, abort_flag, kWaitLimit);
     tc_fence_after();
     const long long qrow = (long long)I * BLK + r;
-    const bool store = ok && r < BLK && qrow < N;
+    const bool store = ok && I < nb && r < BLK && qrow < N;
     __nv_bfloat16* orow = op + ((long long)bh * N + qrow) * D;
-    const float inv_l = (n_kv > 0 && l > 0.f) ? 1.0f / l : 0.f;
+    const float inv_l = (nx > 0 && l > 0.f) ? 1.0f / l : 0.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t raw[32];
-      if (n_kv > 0) {
-        tmem_ld32(tmem + lane_base + C::kO + c * 32, raw);
+      if (nx > 0 && ok) {
+        tmem_ld32(o_addr + c * 32, raw);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -328,7 +403,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (store && lse) {
       // natural-log LSE of the scaled logits: (m + log2 l) * ln 2
-      lse[(long long)bh * N + qrow] = (n_kv > 0) ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      lse[(long long)bh * N + qrow] = (nx > 0) ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
@@ -371,7 +446,7 @@ bool make_map(CUtensorMap* map, const void* base, long long N, int D, long long 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK>
+template <int D, int BLK, int EMU>
 int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
                 const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t st) {
   using C = Cfg<D, BLK>;
@@ -380,20 +455,20 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
       !make_map(&mv, vp, d.N, D, d.BH, BLK))
     return DFS_ERR_CUDA;
   const int max_list = min(kcap, d.nb);
-  size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + (size_t)max_list * sizeof(int32_t);
+  size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + 2 * (size_t)max_list * sizeof(int32_t);
   if (smem > 232448) return DFS_ERR_UNSUPPORTED;
   // Tensor memory per SM is 512 columns: a 512-column CTA must be alone on
   // its SM and a 256-column CTA may share it with one other, so shared
   // memory is padded to make the scheduler place CTAs that way.
   const size_t min_smem = (C::kTmemCols == 512) ? 120 * 1024 : 80 * 1024;
   if (smem < min_smem) smem = min_smem;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, EMU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return DFS_ERR_CUDA;
-  dim3 grid((unsigned)d.nb, (unsigned)d.BH);
+  dim3 grid((unsigned)((d.nb + 1) / 2), (unsigned)d.BH);
   const float scale_log2 = scale * 1.4426950408889634f;
-  attn_fwd_kernel<D, BLK><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb,
-                                                        scale_log2, (__nv_bfloat16*)op, lse, max_list);
+  attn_fwd_kernel<D, BLK, EMU><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb,
+                                                             scale_log2, (__nv_bfloat16*)op, lse, max_list);
   return dfs::launch_status();
 }
 
@@ -411,11 +486,15 @@ extern "C" int dfs_sparse_attn_fwd(const dfs_shape* shape, const void* qp, const
   if (!dfs::aligned16(qp) || !dfs::aligned16(kp) || !dfs::aligned16(vp) || !dfs::aligned16(op) ||
       (lse && !dfs::aligned16(lse)))
     return DFS_ERR_MISALIGNED;
-  if (d.N >= (1LL << 31) || d.BH > 65535 || d.nb > 0x7fffffff) return DFS_ERR_UNSUPPORTED;
+  if (d.N >= (1LL << 31) || d.BH > 65535) return DFS_ERR_UNSUPPORTED;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
   cudaStream_t cs = (cudaStream_t)stream;
-  if (d.D == 128 && d.blk == 128) return launch_attn<128, 128>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
-  if (d.D == 128 && d.blk == 64) return launch_attn<128, 64>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
-  if (d.D == 64 && d.blk == 128) return launch_attn<64, 128>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
-  return launch_attn<64, 64>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+  constexpr int kEmu = DFS_ATTN_EXP2_EMU;
+  if (d.D == 128 && d.blk == 128)
+    return launch_attn<128, 128, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+  if (d.D == 128 && d.blk == 64)
+    return launch_attn<128, 64, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+  if (d.D == 64 && d.blk == 128)
+    return launch_attn<64, 128, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+  return launch_attn<64, 64, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
 }

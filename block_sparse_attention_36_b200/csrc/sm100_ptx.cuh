@@ -12,12 +12,6 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
@@ -36,7 +30,25 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Suspend-time hint (ns) for try_wait: a thread whose phase is not complete
+// may sleep in hardware up to this long instead of spinning, which leaves
+// issue slots to the other warps of its SM sub-partition.
+#ifndef DFS_WAIT_HINT_NS
+#define DFS_WAIT_HINT_NS 0
+#endif
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+#if DFS_WAIT_HINT_NS > 0
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "n"(DFS_WAIT_HINT_NS)
+      : "memory");
+  return ok != 0;
+#else
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -46,36 +58,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+#endif
 }
 
-// Waits for the phase with the given parity to complete. Gives up after
-// limit_ns nanoseconds or when *abort becomes non-zero; returns false then
-// (and raises *abort itself on a timeout).
+// Waits for the phase with the given parity to complete, polling try_wait.
+// Every 64 polls it checks *abort (if given) and the SM clock (a register
+// read); it gives up after limit_cycles cycles or once *abort is set, and
+// returns false then (raising *abort itself on a timeout).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                  uint64_t limit_ns) {
+                                                  long long limit_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
-        *abort = 1;
+      if (abort && *abort) return false;
+      if (clock64() - t0 > limit_cycles) {
+        if (abort) *abort = 1;
         return false;
       }
     }
   }
 }
 
-// Time-bounded wait that ignores the abort flag: used to drain copies and
+// Cycle-bounded wait that ignores the abort flag: used to drain copies and
 // MMAs already issued before a CTA releases its resources.
-__device__ __forceinline__ bool mbar_wait_timed(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
-  }
+__device__ __forceinline__ bool mbar_wait_timed(uint64_t* bar, uint32_t parity, long long limit_cycles) {
+  return mbar_wait_bounded(bar, parity, nullptr, limit_cycles);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -119,8 +128,7 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, one CTA.
@@ -130,8 +138,7 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // Arrives once on *bar when every tcgen05 operation this thread issued so

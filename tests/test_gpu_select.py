@@ -22,7 +22,7 @@ def lib(cuda_device):
 
 
 def _select(lib, scores, shape, params, kcap):
-    B, nh, nb, _ = scores.shape
+    B, nh, nb = shape.B, shape.nh, shape.nb
     idx = torch.full((B, nh, nb, kcap), -7, dtype=torch.int32, device="cuda")
     cnt = torch.full((B, nh, nb), -7, dtype=torch.int32, device="cuda")
     sc = None if scores is None else torch.from_numpy(np.ascontiguousarray(scores, dtype=np.float32)).cuda()
