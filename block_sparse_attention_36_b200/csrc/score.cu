@@ -200,3 +200,78 @@ extern "C" int dfs_block_score(const dfs_shape* shape, const void* qp, const voi
   }
   return dfs::launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// dfs_block_score_noalloc: the same two kernels, with the pooled means kept
+// in a buffer compiled into the library instead of a caller workspace, for
+// callers that cannot allocate device memory (see include/dfsattn.h).
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = DFS_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DFS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DFS_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DFS_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return DFS_OK;
+}
+
+}  // namespace
+
+extern "C" int dfs_block_score_noalloc(const dfs_shape* shape, const void* qp, const void* kp, float scale,
+                                       float* scores, dfs_stream_t stream) {
+  dfs::Dims d;
+  int st = dfs::check_shape(shape, &d, true);
+  if (st != DFS_OK) return st;
+  if (!qp || !kp || !scores) return DFS_ERR_INVALID_ARG;
+  if (!dfs::aligned16(qp) || !dfs::aligned16(kp) || !dfs::aligned16(scores)) return DFS_ERR_MISALIGNED;
+  const size_t need = (size_t)2 * d.BH * d.nsb * d.D * sizeof(float);
+  if (need > kNoallocScratchBytes) return DFS_ERR_WORKSPACE;   // beyond the built-in buffer
+  if (d.BH > 65535) return DFS_ERR_UNSUPPORTED;
+  float* pooled = nullptr;
+  st = noalloc_scratch(&pooled);
+  if (st != DFS_OK) return st;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
+  cudaStream_t cs = (cudaStream_t)stream;
+  // Every pooled value the score kernel reads is written first by the pool
+  // kernel on the same stream, so the buffer needs no clearing.
+  const long long jobs = d.BH * d.nsb;
+  dim3 pg((unsigned)((jobs + 7) / 8), 2);
+  if (d.D == 128)
+    pool_kernel<128><<<pg, 256, 0, cs>>>((const __nv_bfloat16*)qp, (const __nv_bfloat16*)kp, pooled,
+                                         d.N, d.sb, d.nsb, d.BH);
+  else
+    pool_kernel<64><<<pg, 256, 0, cs>>>((const __nv_bfloat16*)qp, (const __nv_bfloat16*)kp, pooled,
+                                        d.N, d.sb, d.nsb, d.BH);
+  st = dfs::launch_status();
+  if (st != DFS_OK) return st;
+  const float* qbar = pooled;
+  const float* kbar = pooled + d.BH * d.nsb * d.D;
+  const unsigned tiles = (unsigned)((d.nsb + kTile - 1) / kTile);
+  dim3 sg(tiles, tiles, (unsigned)d.BH);
+  switch (d.r) {
+    case 1: score_kernel<1><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+    case 2: score_kernel<2><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+    case 4: score_kernel<4><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+    default: score_kernel<8><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+  }
+  return dfs::launch_status();
+}

@@ -41,7 +41,7 @@ MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_L
 # C entry points declared in include/dfsattn.h.
 EXPORTS = (
     "dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd", "dfs_unperm",
-    "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version",
+    "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version", "dfs_block_score_noalloc",
 )
 
 
@@ -64,6 +64,7 @@ def _load():
     lib.dfs_hilbert_perm.argtypes = [sp, I, P, P, I, P, P, P, P, P, P, P]
     lib.dfs_block_score.argtypes = [sp, P, P, F, P, P, S, P]
     lib.dfs_select_mask.argtypes = [sp, P, ctypes.POINTER(_SelectParams), P, P, I, P]
+    lib.dfs_block_score_noalloc.argtypes = [sp, P, P, F, P, P]
     lib.dfs_sparse_attn_fwd.argtypes = [sp, P, P, P, P, P, I, F, P, P, P]
     lib.dfs_unperm.argtypes = [sp, P, P, P, P]
     lib.dfs_workspace_bytes.argtypes = [sp, I]
@@ -73,7 +74,7 @@ def _load():
     lib.dfs_status_string.restype = ctypes.c_char_p
     lib.dfs_version.argtypes = []
     for name in ("dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd",
-                 "dfs_unperm", "dfs_get_error_flags", "dfs_version"):
+                 "dfs_unperm", "dfs_get_error_flags", "dfs_version", "dfs_block_score_noalloc"):
         getattr(lib, name).restype = I
     return lib
 
@@ -147,6 +148,18 @@ def dfs_block_score(shape: Shape, qp, kp, scale, scores, ws, stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("dfs_block_score", LIB.dfs_block_score(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), float(scale), _ptr(scores), _ptr(ws), nbytes, _stream(stream)))
+
+
+def dfs_block_score_noalloc(shape: Shape, qp, kp, scale, scores, stream=None):
+    """dfs_block_score with the library's built-in scratch buffer instead of a
+    workspace, for callers that cannot allocate device memory (see the C
+    header for the size limit, first-call set-up and the sharing rule)."""
+    sh = shape.c()
+    _check("dfs_block_score_noalloc", LIB.dfs_block_score_noalloc(
+        ctypes.byref(sh), _ptr(qp), _ptr(kp), float(scale), _ptr(scores), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def select_params(mode, k=0, cap=0, tau=0.0, lvsa_T_per=8, lvsa_C=21, lvsa_step=0):

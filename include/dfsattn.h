@@ -126,6 +126,29 @@ int dfs_hilbert_perm(const dfs_shape *shape, int order, int32_t *perm, int32_t *
 int dfs_block_score(const dfs_shape *shape, const void *qp, const void *kp, float scale,
                     float *scores, void *ws, size_t ws_bytes, dfs_stream_t stream);
 
+/* dfs_block_score_noalloc -- dfs_block_score without a caller workspace.
+ *
+ * Not from the pages (they have no counterpart): an entry point for callers
+ * that cannot allocate device memory -- for example a plugin whose host
+ * hands it only tensors and a stream, or a serving process whose caching
+ * allocator has already reserved the device, where a raw cudaMalloc would
+ * fail or stall the stream. Same arguments, arithmetic and output as
+ * dfs_block_score, but the pooled means live in a buffer compiled into the
+ * library: DFS_NOALLOC_SCRATCH_BYTES bytes of device memory, held by every
+ * GPU that loads the library until the process exits. A shape that needs
+ * more (2 * B * nh * ceil(N / sb) * D * 4 bytes) returns DFS_ERR_WORKSPACE
+ * without launching. The call allocates nothing; the first call on a device
+ * looks the buffer's device address up once (cudaGetSymbolAddress) with
+ * that device current, so make that first call before any stream capture.
+ * All calls in the process share the one buffer and it keeps the last
+ * call's contents (each call writes every value it later reads, so nothing
+ * needs clearing): calls that may overlap on the GPU -- on different
+ * streams, or from different threads -- race and must be serialised by the
+ * caller.                                                                  */
+#define DFS_NOALLOC_SCRATCH_BYTES (32u << 20)
+int dfs_block_score_noalloc(const dfs_shape *shape, const void *qp, const void *kp, float scale,
+                            float *scores, dfs_stream_t stream);
+
 /* dfs_select_mask -- key-block selection (DFSAttn, Methodology item 3;
  * VMoBA abstract, modification 3; LVSA section 2).
  *
