@@ -91,7 +91,7 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t d
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint64_t oa = (uint64_t)(((kk >> 2) * (kQRows * 128) + (kk & 3) * 32) >> 4);
     const uint64_t ob = (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
-    mma_ss(d_tmem, dq + oa, dk + ob, idesc, kk > 0 ? 1u : 0u);
+    mma_ss_warp(d_tmem, dq + oa, dk + ob, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -102,7 +102,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
   constexpr uint32_t idesc = idesc_bf16_f32(kQRows, D, 1);
 #pragma unroll
   for (int kk = 0; kk < BLK / 16; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_warp(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, int BLK, int EMU>
@@ -173,15 +173,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp < 4) {
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensor_map(&tm_q);
-      prefetch_tensor_map(&tm_k);
-      prefetch_tensor_map(&tm_v);
+    // Warp-uniform loop; elect.sync picks the lane that arms a barrier or
+    // issues a copy.
+    {
+      if (lane == 0) {
+        prefetch_tensor_map(&tm_q);
+        prefetch_tensor_map(&tm_k);
+        prefetch_tensor_map(&tm_v);
+      }
       for (int x = 0; x < 2; ++x) {
         if (n[x] == 0) continue;
-        mbar_arrive_expect_tx(&bars->q_full[x], C::kQBytes);
+        mbar_arrive_expect_tx_warp(&bars->q_full[x], C::kQBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(smem + C::kQOff + x * C::kQBytes + c * (kQRows * 128), &tm_q, &bars->q_full[x], c * 64,
+          tma_load_3d_warp(smem + C::kQOff + x * C::kQBytes + c * (kQRows * 128), &tm_q, &bars->q_full[x], c * 64,
                       (I0 + x) * BLK, bh);
       }
       // Same step order as the MMA issuer: step -1 loads K_A(0), K_B(0); step
@@ -202,13 +206,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&bars->kv_full[st], C::kTileBytes);
+            mbar_arrive_expect_tx_warp(&bars->kv_full[st], C::kTileBytes);
             const int J = lists[x * max_list + jj];
             uint8_t* dst = smem + C::kRingOff + st * C::kTileBytes;
             const CUtensorMap* map = kind == 0 ? &tm_v : &tm_k;
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(dst + c * (BLK * 128), map, &bars->kv_full[st], c * 64, J * BLK, bh);
+              tma_load_3d_warp(dst + c * (BLK * 128), map, &bars->kv_full[st], c * 64, J * BLK, bh);
             ++t;
           }
           if (!ok) break;
@@ -223,7 +227,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop (warp-uniform control flow and
+    // operands); elect.sync inside each MMA / commit picks the issuing lane.
+    {
       // Descriptors are built once; a K step or a ring stage only moves the
       // start-address field (16-byte units), so each MMA costs an add.
       const uint64_t dq = desc_sw128(smem_addr(smem + C::kQOff), 16, 1024);
@@ -250,7 +256,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
             issue_pv<D, BLK>(tmem + C::o_col(x), tmem + C::s_col(x), dv + (uint64_t)((st * C::kTileBytes) >> 4),
                              step > 0);
-            mma_commit(&bars->kv_empty[st]);
+            mma_commit_warp(&bars->kv_empty[st]);
             ++t;
           }
           if (step + 1 < nx) {
@@ -258,16 +264,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
             issue_s<D, BLK>(tmem + C::s_col(x), dq + (uint64_t)((x * C::kQBytes) >> 4),
                             dk + (uint64_t)((st * C::kTileBytes) >> 4));
-            mma_commit(&bars->s_full[x]);
-            mma_commit(&bars->kv_empty[st]);
+            mma_commit_warp(&bars->s_full[x]);
+            mma_commit_warp(&bars->kv_empty[st]);
             ++t;
           } else if (step >= 0) {
-            mma_commit(&bars->o_final[x]);
+            mma_commit_warp(&bars->o_final[x]);
           }
         }
       }
       // Every MMA must finish before tensor memory is released.
-      mma_commit(&bars->mma_done);
+      mma_commit_warp(&bars->mma_done);
       mbar_wait_timed(&bars->mma_done, 0, kDrainLimit);
     }
     __syncwarp();
