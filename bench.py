@@ -39,6 +39,28 @@ METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
 KERNELS_PER_STEP = {"topk": 8, "threshold": 8, "lvsa": 6}   # 3 gathers, pool, score, select, attn, scatter
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per attention launch from one ncu capture
+# (profiles/attn_fwd_<workload>.md), valid only for the attention sources
+# whose hash is recorded with it; reported as null once they change.
+ATTN_TRAFFIC = {"wan_1p3b_layer": (297_903_360 + 82_006_784, "008d78ef19061aff")}
+ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh")
+
+
+def attn_sources_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_attention_36_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def attn_traffic(workload):
+    entry = ATTN_TRAFFIC.get(workload)
+    if entry is None or entry[1] != attn_sources_hash():
+        return None
+    return entry[0]
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -180,7 +202,7 @@ def run_ours(args):
     rank, world, local = dist_setup(args.gpus)
     wl = synth.WORKLOADS[args.workload]
     if wl.mode == "schedule":
-        raise SystemExit("the schedule workload is timed by --workload wan_schedule_50 via run_schedule")
+        return run_schedule(args, wl, rank, world, local)
     qkv = synth.workload_inputs(wl, seed=args.seed + rank)
     q, k, v = (qkv[n].cuda() for n in ("q", "k", "v"))
     layer, kk, cap = make_layer(bsa, wl)
@@ -252,7 +274,7 @@ def run_ours(args):
         peak = float(peaks["bf16_tflops"])
         ms_step = ms_total_max / args.steps
         value = flops_all / (ms_total_max * 1e-3) / 1e12
-        traffic = None
+        traffic = attn_traffic(wl.name)
         line = {
             "metric": METRIC,
             "value": round(value, 3),
@@ -284,6 +306,79 @@ def run_ours(args):
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(wl, qkv, kk, cap, budget_s=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_schedule(args, wl, rank, world, local):
+    """The 50-step denoising loop: Q/K change every step (V is fixed), the
+    keep budget falls from 40 % to 10 %, masks are rebuilt every 5 steps and
+    attention runs every step. Reports the amortised time per step and the
+    kept-block TFLOP/s over all 50 steps."""
+    import torch
+    import synth
+    import block_sparse_attention_36_b200 as bsa
+    from block_sparse_attention_36_b200 import dfsattn
+    from block_sparse_attention_36_b200 import schedule
+
+    s = bsa.Shape(wl.B, wl.nh, wl.D, wl.T, wl.H, wl.W, wl.blk, wl.sb)
+    kmax = schedule.keep_budget(0, s.nb, wl.n_steps, wl.refresh)
+    layer = bsa.DfsLayer(s, order=wl.order, mode="topk", k=kmax, kcap=kmax)
+    fields = {n: t.cuda() for n, t in synth.schedule_fields(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=args.seed + rank).items()}
+    v = synth.field_qkv(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=args.seed + rank, which=("v",))["v"].cuda()
+    steps_qk = [synth.schedule_qk_device(fields, st, seed=args.seed + rank, n_steps=wl.n_steps)
+                for st in range(wl.n_steps)]
+    del fields
+    stream = torch.cuda.current_stream()
+
+    def run_loop(count_flops=False):
+        flops = 0.0
+        for st in range(wl.n_steps):
+            refresh = schedule.is_refresh(st, wl.refresh)
+            if refresh:
+                layer.set_budget(k=schedule.keep_budget(st, s.nb, wl.n_steps, wl.refresh))
+            layer.forward(steps_qk[st]["q"], steps_qk[st]["k"], v, refresh_mask=refresh)
+            if count_flops:
+                torch.cuda.synchronize()
+                flops += 4.0 * wl.D * layer.kept_pairs()
+        return flops
+
+    flops_loop = run_loop(count_flops=True)       # also the first warm-up pass
+    for _ in range(max(0, args.warmup - 1)):
+        run_loop()
+    torch.cuda.synchronize()
+    assert dfsattn.dfs_get_error_flags(clear=True) == 0
+    reps = max(1, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        run_loop()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_step = ms / (reps * wl.n_steps)
+    flops_all = sum_over_ranks(flops_loop * reps, world)
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(flops_all / (ms * 1e-3) / 1e12, 3),
+                "unit": "TFLOP/s (kept-block, amortised over the 50-step loop)", "n_gpus": world,
+                "steps": reps * wl.n_steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded fields; per-step noise drawn on the device)",
+                "config": {"workload": (f"{wl.name}: B={wl.B} nh={wl.nh} D={wl.D} grid {wl.T}x{wl.H}x{wl.W} "
+                                        f"(N={wl.N}), {wl.n_steps} steps, top-k 103 -> 32 of {s.nb}, "
+                                        f"mask refresh every {wl.refresh} steps, attention every step"),
+                           "parallelism": f"replicas x{world}"},
+                "gpu_launches": None, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -137,6 +137,38 @@ def schedule_qk(T, H, W, nh, D, s, B=1, seed=0, n_steps=50, threads=8):
     return out
 
 
+def schedule_fields(T, H, W, nh, D, B=1, seed=0, threads=8):
+    """The noise-free, normalised Q and K fields of the schedule workload,
+    fp32 CPU tensors [B, N, nh, D] (the part of the recipe shared by all steps)."""
+    N = T * H * W
+    out = {n: torch.empty((B, N, nh, D), dtype=torch.float32) for n in ("q", "k")}
+
+    def one(j):
+        b, name, h = j
+        rng = np.random.default_rng([seed, b, TENSOR_IDS[name], h])
+        return torch.from_numpy(_normalise(_smooth_field(rng, T, H, W, D)).astype(np.float32))
+
+    jobs = [(b, name, h) for name in ("q", "k") for b in range(B) for h in range(nh)]
+    with ThreadPoolExecutor(max_workers=max(1, threads)) as ex:
+        res = list(ex.map(one, jobs))
+    for (b, name, h), x in zip(jobs, res):
+        out[name][b, :, h, :] = x
+    return out
+
+
+def schedule_qk_device(fields, s, seed=0, n_steps=50):
+    """Q, K of step s for timing runs: the same recipe as schedule_qk, but
+    eps_s is drawn on the fields' device by torch's generator seeded with
+    (seed, s) -- the same distribution, a different realisation. Parity tests
+    use schedule_qk."""
+    dev = fields["q"].device
+    g = torch.Generator(device=dev)
+    g.manual_seed(1_000_003 * (seed + 1) + s)
+    sig = schedule_sigma(s, n_steps)
+    return {n: (fields[n] + sig * torch.randn(fields[n].shape, generator=g, device=dev)).to(torch.bfloat16)
+            for n in ("q", "k")}
+
+
 # ---------------------------------------------------------------------------
 # The five workloads (shapes, block sizes and selection settings).
 # ---------------------------------------------------------------------------
