@@ -36,7 +36,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
-KERNELS_PER_STEP = {"topk": 8, "threshold": 8, "lvsa": 6}   # 3 gathers, pool, score, select, attn, scatter
+# fused gather + pooling (1 launch), score, select, attention, scatter; LVSA: 3 gathers, select, attention, scatter
+KERNELS_PER_STEP = {"topk": 5, "threshold": 5, "lvsa": 6}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per attention launch from one ncu capture
@@ -229,8 +230,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     start.record(stream)
     for i in range(args.steps):
-        layer.permute(q, k, v)
-        layer.build_mask()
+        layer.prepare(q, k, v)
         ev_attn[i][0].record(stream)
         dfsattn.dfs_sparse_attn_fwd(layer.shape, layer.qp, layer.kp, layer.vp, layer.kv_idx, layer.kv_cnt,
                                     layer.kcap, layer.scale, layer.op, None)

@@ -208,6 +208,66 @@ int launch_copy(bool to_curve, const void* src, void* dst, const int32_t* perm, 
   return dfs::launch_status();
 }
 
+// Gather of Q, K, V into curve order fused with the sub-block means of Q and
+// K. One CTA per (sub-block j, batch b, tensor): thread v owns one 16-byte
+// column (head h, eight dims) and walks the sub-block's tokens in order, so
+// the column sum needs no cross-thread reduction; loads of eight tokens are
+// in flight per thread. pooled: fp32 [2, B, nh, nsb, D] (Q then K).
+template <int D>
+__global__ void __launch_bounds__(512)
+gather_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+                   uint4* __restrict__ qp, uint4* __restrict__ kp, uint4* __restrict__ vp,
+                   const int32_t* __restrict__ perm, float* __restrict__ pooled, int N, int nh, int sb, int nsb,
+                   int B) {
+  constexpr int kDvec = D / 8;
+  const int vpt = nh * kDvec;
+  const int col = threadIdx.x;
+  if (col >= vpt) return;
+  const int j = blockIdx.x, b = blockIdx.y, tsel = blockIdx.z;  // tensor: 0 Q, 1 K, 2 V
+  const uint4* src = tsel == 0 ? q : (tsel == 1 ? k : v);
+  uint4* dst = tsel == 0 ? qp : (tsel == 1 ? kp : vp);
+  if (!src) return;
+  const int h = col / kDvec, d8 = col - h * kDvec;
+  const int i0 = j * sb, i1 = min(i0 + sb, N);
+  const uint4* s_base = src + (long long)b * N * vpt + col;
+  uint4* d_base = dst + ((long long)(b * nh + h) * N) * kDvec + d8;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int i = i0; i < i1; i += 8) {
+    uint4 val[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int ii = i + u;
+      if (ii < i1) val[u] = __ldg(s_base + (long long)__ldg(perm + ii) * vpt);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int ii = i + u;
+      if (ii < i1) {
+        d_base[(long long)ii * kDvec] = val[u];
+        if (tsel < 2) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&val[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            acc[2 * e] += f.x;
+            acc[2 * e + 1] += f.y;
+          }
+        }
+      }
+    }
+  }
+  if (tsel < 2) {
+    const float fc = (float)(i1 - i0);
+    float* out = pooled + ((((long long)tsel * B + b) * nh + h) * nsb + j) * D + d8 * 8;
+    reinterpret_cast<float4*>(out)[0] =
+        make_float4(__fdiv_rn(acc[0], fc), __fdiv_rn(acc[1], fc), __fdiv_rn(acc[2], fc), __fdiv_rn(acc[3], fc));
+    reinterpret_cast<float4*>(out)[1] =
+        make_float4(__fdiv_rn(acc[4], fc), __fdiv_rn(acc[5], fc), __fdiv_rn(acc[6], fc), __fdiv_rn(acc[7], fc));
+  }
+}
+
 }  // namespace
 
 DFS_DEFINE_FLAG_READER(dfs_detail_flags_perm, g_perm_flags)
@@ -250,4 +310,43 @@ extern "C" int dfs_unperm(const dfs_shape* shape, const int32_t* perm, const voi
   if (!perm || !op || !o) return DFS_ERR_INVALID_ARG;
   if (!dfs::aligned16(op) || !dfs::aligned16(o)) return DFS_ERR_MISALIGNED;
   return launch_copy(false, op, o, perm, d, (cudaStream_t)stream);
+}
+
+extern "C" int dfs_hilbert_perm_pooled(const dfs_shape* shape, int order, int32_t* perm, int32_t* inv,
+                                       int build_index, const void* q, const void* k, const void* v, void* qp,
+                                       void* kp, void* vp, void* ws, size_t ws_bytes, dfs_stream_t stream) {
+  dfs::Dims d;
+  int st = dfs::check_shape(shape, &d, true);
+  if (st != DFS_OK) return st;
+  if (order != DFS_ORDER_RASTER && order != DFS_ORDER_HILBERT3D) return DFS_ERR_INVALID_ARG;
+  if (!perm || (build_index && !inv)) return DFS_ERR_INVALID_ARG;
+  if (!q || !k || !qp || !kp) return DFS_ERR_INVALID_ARG;
+  if ((v == nullptr) != (vp == nullptr)) return DFS_ERR_INVALID_ARG;
+  const void* ptrs[6] = {q, k, v, qp, kp, vp};
+  for (const void* p : ptrs)
+    if (p && !dfs::aligned16(p)) return DFS_ERR_MISALIGNED;
+  const size_t need = (size_t)2 * d.BH * d.nsb * d.D * sizeof(float);
+  if (!ws || ws_bytes < need) return DFS_ERR_WORKSPACE;
+  if (!dfs::aligned16(ws)) return DFS_ERR_MISALIGNED;
+  const int vpt = d.nh * (d.D / 8);
+  if (vpt > 512 || d.B > 65535 || d.N >= (1LL << 31)) return DFS_ERR_UNSUPPORTED;
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (build_index) {
+    const int threads = 256;
+    const long long grid = (d.N + threads - 1) / threads;
+    hilbert_index_kernel<<<(unsigned)grid, threads, 0, cs>>>(d.T, d.H, d.W, order, perm, inv);
+    st = dfs::launch_status();
+    if (st != DFS_OK) return st;
+  }
+  const int threads = ((vpt + 31) / 32) * 32;
+  dim3 grid((unsigned)d.nsb, (unsigned)d.B, v ? 3u : 2u);
+  if (d.D == 128)
+    gather_pool_kernel<128><<<grid, threads, 0, cs>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (uint4*)qp,
+                                                      (uint4*)kp, (uint4*)vp, perm, (float*)ws, (int)d.N, d.nh,
+                                                      d.sb, d.nsb, d.B);
+  else
+    gather_pool_kernel<64><<<grid, threads, 0, cs>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, (uint4*)qp,
+                                                     (uint4*)kp, (uint4*)vp, perm, (float*)ws, (int)d.N, d.nh,
+                                                     d.sb, d.nsb, d.B);
+  return dfs::launch_status();
 }

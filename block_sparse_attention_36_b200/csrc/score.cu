@@ -201,6 +201,32 @@ extern "C" int dfs_block_score(const dfs_shape* shape, const void* qp, const voi
   return dfs::launch_status();
 }
 
+extern "C" int dfs_block_score_pooled(const dfs_shape* shape, float scale, float* scores, const void* ws,
+                                      size_t ws_bytes, dfs_stream_t stream) {
+  dfs::Dims d;
+  int st = dfs::check_shape(shape, &d, true);
+  if (st != DFS_OK) return st;
+  if (!scores) return DFS_ERR_INVALID_ARG;
+  if (!dfs::aligned16(scores)) return DFS_ERR_MISALIGNED;
+  const size_t need = (size_t)2 * d.BH * d.nsb * d.D * sizeof(float);
+  if (!ws || ws_bytes < need) return DFS_ERR_WORKSPACE;
+  if (!dfs::aligned16(ws)) return DFS_ERR_MISALIGNED;
+  if (d.BH > 65535) return DFS_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
+  cudaStream_t cs = (cudaStream_t)stream;
+  const float* qbar = (const float*)ws;
+  const float* kbar = qbar + d.BH * d.nsb * d.D;
+  const unsigned tiles = (unsigned)((d.nsb + kTile - 1) / kTile);
+  dim3 sg(tiles, tiles, (unsigned)d.BH);
+  switch (d.r) {
+    case 1: score_kernel<1><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+    case 2: score_kernel<2><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+    case 4: score_kernel<4><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+    default: score_kernel<8><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
+  }
+  return dfs::launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // dfs_block_score_noalloc: the same two kernels, with the pooled means kept
 // in a buffer compiled into the library instead of a caller workspace, for

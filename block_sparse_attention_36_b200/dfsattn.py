@@ -42,6 +42,7 @@ MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_L
 EXPORTS = (
     "dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd", "dfs_unperm",
     "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version", "dfs_block_score_noalloc",
+    "dfs_hilbert_perm_pooled", "dfs_block_score_pooled",
 )
 
 
@@ -65,6 +66,8 @@ def _load():
     lib.dfs_block_score.argtypes = [sp, P, P, F, P, P, S, P]
     lib.dfs_select_mask.argtypes = [sp, P, ctypes.POINTER(_SelectParams), P, P, I, P]
     lib.dfs_block_score_noalloc.argtypes = [sp, P, P, F, P, P]
+    lib.dfs_hilbert_perm_pooled.argtypes = [sp, I, P, P, I, P, P, P, P, P, P, P, S, P]
+    lib.dfs_block_score_pooled.argtypes = [sp, F, P, P, S, P]
     lib.dfs_sparse_attn_fwd.argtypes = [sp, P, P, P, P, P, I, F, P, P, P]
     lib.dfs_unperm.argtypes = [sp, P, P, P, P]
     lib.dfs_workspace_bytes.argtypes = [sp, I]
@@ -74,7 +77,8 @@ def _load():
     lib.dfs_status_string.restype = ctypes.c_char_p
     lib.dfs_version.argtypes = []
     for name in ("dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd",
-                 "dfs_unperm", "dfs_get_error_flags", "dfs_version", "dfs_block_score_noalloc"):
+                 "dfs_unperm", "dfs_get_error_flags", "dfs_version", "dfs_block_score_noalloc",
+                 "dfs_hilbert_perm_pooled", "dfs_block_score_pooled"):
         getattr(lib, name).restype = I
     return lib
 
@@ -136,6 +140,22 @@ def dfs_hilbert_perm(shape: Shape, order, perm, inv, build_index, q, k, v, qp, k
     _check("dfs_hilbert_perm", LIB.dfs_hilbert_perm(
         ctypes.byref(sh), int(order), _ptr(perm), _ptr(inv), int(bool(build_index)),
         _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp), _stream(stream)))
+
+
+def dfs_hilbert_perm_pooled(shape: Shape, order, perm, inv, build_index, q, k, v, qp, kp, vp, ws, stream=None):
+    order = ORDERS.get(order, order)
+    sh = shape.c()
+    _check("dfs_hilbert_perm_pooled", LIB.dfs_hilbert_perm_pooled(
+        ctypes.byref(sh), int(order), _ptr(perm), _ptr(inv), int(bool(build_index)),
+        _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def dfs_block_score_pooled(shape: Shape, scale, scores, ws, stream=None):
+    sh = shape.c()
+    _check("dfs_block_score_pooled", LIB.dfs_block_score_pooled(
+        ctypes.byref(sh), float(scale), _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def dfs_workspace_bytes(shape: Shape, which=DFS_WS_BLOCK_SCORE) -> int:

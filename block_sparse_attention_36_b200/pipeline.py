@@ -52,6 +52,8 @@ class DfsLayer:
             self.scores = None
             self.ws = None
         self._index_built = False
+        # the fused reorder + pooling needs nh * D / 8 <= 512
+        self.fused_pool = s.nh * s.D // 8 <= 512
 
     def set_budget(self, k=None, cap=None, tau=None, lvsa_step=None):
         p = self.params
@@ -82,11 +84,28 @@ class DfsLayer:
                                 self.scale, self.op, self.lse, stream)
         lib.dfs_unperm(self.shape, self.perm, self.op, self.out, stream)
 
+    def permute_pooled(self, q, k, v, stream=None):
+        """Reorder Q, K, V and pool Q, K into the score workspace in one pass."""
+        lib.dfs_hilbert_perm_pooled(self.shape, self.order, self.perm, self.inv, not self._index_built, q, k, v,
+                                    self.qp, self.kp, self.vp, self.ws, stream)
+        self._index_built = True
+
+    def prepare(self, q, k, v, refresh_mask=True, stream=None):
+        """Reorder Q, K, V and, if asked, rebuild the mask. When the mask is
+        rebuilt from scores, the reorder also pools Q and K (one pass over the
+        data) and scoring starts from those means."""
+        if refresh_mask and self.mode != "lvsa" and self.fused_pool:
+            self.permute_pooled(q, k, v, stream)
+            lib.dfs_block_score_pooled(self.shape, self.scale, self.scores, self.ws, stream)
+            lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
+        else:
+            self.permute(q, k, v, stream)
+            if refresh_mask:
+                self.build_mask(stream)
+
     def forward(self, q, k, v, refresh_mask=True, stream=None):
         """q, k, v: bf16 [B, N, nh, D] on the device (raster order). Returns the output buffer."""
-        self.permute(q, k, v, stream)
-        if refresh_mask:
-            self.build_mask(stream)
+        self.prepare(q, k, v, refresh_mask, stream)
         self.attend(stream)
         return self.out
 

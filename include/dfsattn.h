@@ -126,6 +126,26 @@ int dfs_hilbert_perm(const dfs_shape *shape, int order, int32_t *perm, int32_t *
 int dfs_block_score(const dfs_shape *shape, const void *qp, const void *kp, float scale,
                     float *scores, void *ws, size_t ws_bytes, dfs_stream_t stream);
 
+/* dfs_hilbert_perm_pooled -- dfs_hilbert_perm fused with the first half of
+ * dfs_block_score (DFSAttn, Methodology items 1 and 2).
+ *
+ * Same reorder as dfs_hilbert_perm (q, k, qp, kp required; v and vp both
+ * NULL or both given), and in the same pass over the data it writes the
+ * sub-block means of the reordered Q and K to ws, fp32 [2, B, nh, nsb, D]
+ * (the layout dfs_block_score keeps in its workspace; ws_bytes >=
+ * dfs_workspace_bytes(shape, DFS_WS_BLOCK_SCORE)). Needs nh * D / 8 <= 512.
+ * Follow it with dfs_block_score_pooled on the same ws.                    */
+int dfs_hilbert_perm_pooled(const dfs_shape *shape, int order, int32_t *perm, int32_t *inv,
+                            int build_index, const void *q, const void *k, const void *v,
+                            void *qp, void *kp, void *vp, void *ws, size_t ws_bytes,
+                            dfs_stream_t stream);
+
+/* dfs_block_score_pooled -- the second half of dfs_block_score: block scores
+ * from sub-block means already in ws (as dfs_hilbert_perm_pooled writes
+ * them); same scale rule and output as dfs_block_score.                   */
+int dfs_block_score_pooled(const dfs_shape *shape, float scale, float *scores, const void *ws,
+                           size_t ws_bytes, dfs_stream_t stream);
+
 /* dfs_block_score_noalloc -- dfs_block_score without a caller workspace.
  *
  * Not from the pages (they have no counterpart): an entry point for callers

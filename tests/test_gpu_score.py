@@ -67,3 +67,40 @@ def test_explicit_scale(lib):
     qp, kp, got, _, s = _run(lib, 1, 1, 64, 500, 64, 16, seed=3, scale=0.5)
     ref = scoring.block_scores(qp.double().numpy(), kp.double().numpy(), 64, 16, 0.5)
     assert np.abs(got - ref).max() < 1e-4
+
+
+@pytest.mark.parametrize("B,nh,D,grid,blk,sb", [(1, 2, 64, (8, 16, 16), 64, 16), (2, 3, 128, (3, 7, 11), 128, 32),
+                                                (1, 12, 128, (21, 30, 52), 128, 32), (1, 1, 128, (1, 1, 100), 64, 8)])
+def test_fused_gather_pool_then_score(lib, B, nh, D, grid, blk, sb):
+    """dfs_hilbert_perm_pooled reorders exactly like the oracle and writes the
+    sub-block means; dfs_block_score_pooled turns them into block scores."""
+    from oracle import hilbert
+    T, H, W = grid
+    N = T * H * W
+    g = torch.Generator().manual_seed(N + D)
+    x = [torch.randn((B, N, nh, D), generator=g).to(torch.bfloat16) for _ in range(3)]
+    s = lib.Shape(B, nh, D, T, H, W, blk, sb)
+    perm = torch.empty(N, dtype=torch.int32, device="cuda")
+    inv = torch.empty_like(perm)
+    xp = [torch.empty((B, nh, N, D), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    ws = torch.empty(lib.dfs_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    scores = torch.empty((B, nh, s.nb, s.nb), dtype=torch.float32, device="cuda")
+    lib.dfs_hilbert_perm_pooled(s, "hilbert3d", perm, inv, 1, *(t.cuda() for t in x), *xp, ws)
+    lib.dfs_block_score_pooled(s, 0.0, scores, ws)
+    torch.cuda.synchronize()
+    operm, _ = hilbert.hilbert_perm(T, H, W)
+    assert np.array_equal(perm.cpu().numpy(), operm)
+    ref = [hilbert.permute_tokens(t.view(torch.int16).numpy(), operm) for t in x]
+    for t in range(3):
+        assert np.array_equal(xp[t].cpu().view(torch.int16).numpy(), ref[t])
+    q64 = hilbert.permute_tokens(x[0].double().numpy(), operm)
+    k64 = hilbert.permute_tokens(x[1].double().numpy(), operm)
+    pooled = ws.view(torch.float32)[: 2 * B * nh * s.nsb * D].view(2, B, nh, s.nsb, D).cpu().numpy()
+    oq, ok = scoring.pool_subblocks(q64, sb), scoring.pool_subblocks(k64, sb)
+    tol_pool = (sb + 2) * U32 * max(np.abs(q64).max(), np.abs(k64).max())
+    assert np.abs(pooled[0] - oq).max() <= tol_pool
+    assert np.abs(pooled[1] - ok).max() <= tol_pool
+    scale = 1.0 / math.sqrt(D)
+    ref_s = scoring.block_scores(q64, k64, blk, sb, scale)
+    mag = scale * D * np.abs(oq).max() * np.abs(ok).max()
+    assert np.abs(scores.cpu().numpy() - ref_s).max() <= (D + 2 * sb + 4) * U32 * mag
