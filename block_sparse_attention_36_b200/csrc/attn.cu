@@ -310,14 +310,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int e = 0; e < BLK; ++e)
           if (e >= rem) sv[e] = -INFINITY;
       }
-      // row maximum, eight independent chains
+      // row maximum: eight independent chains of three-input maxima
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
 #pragma unroll
-      for (int e = 8; e < BLK; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], sv[e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int e = 8; e + 16 <= BLK; e += 16)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], sv[e + c], sv[e + 8 + c]);
+      if ((BLK - 8) % 16 != 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(mx8[c], sv[BLK - 8 + c]);
+      }
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       const float m_blk = mx * scale_log2;
       bool rescale = false;
       float m_use;
