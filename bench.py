@@ -228,8 +228,14 @@ def run_ours(args):
         time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
+    graph = layer.capture_graph(q, k, v) if args.graph else None
+    barrier(world)
+    torch.cuda.synchronize()
     start.record(stream)
     for i in range(args.steps):
+        if graph is not None:
+            graph.replay()
+            continue
         layer.prepare(q, k, v)
         ev_attn[i][0].record(stream)
         dfsattn.dfs_sparse_attn_fwd(layer.shape, layer.qp, layer.kp, layer.vp, layer.kv_idx, layer.kv_cnt,
@@ -241,6 +247,15 @@ def run_ours(args):
     barrier(world)
     clk = clocks.stop() if clocks else None
     ms_total = start.elapsed_time(stop)
+    if graph is not None:
+        # attention-kernel time from eager launches (events cannot sit inside the graph replay)
+        for i in range(args.steps):
+            ev_attn[i][0].record(stream)
+            dfsattn.dfs_sparse_attn_fwd(layer.shape, layer.qp, layer.kp, layer.vp, layer.kv_idx, layer.kv_cnt,
+                                        layer.kcap, layer.scale, layer.op, None)
+            ev_attn[i][1].record(stream)
+        torch.cuda.synchronize()
+        del graph
     attn_ms = [a.elapsed_time(b) for a, b in ev_attn]
     ms_total_max = max_over_ranks(ms_total, world)
     flops_all = sum_over_ranks(flops_step * args.steps, world)
@@ -293,7 +308,8 @@ def run_ours(args):
             "config": {"workload": workload_config(wl, kk, cap), "kept_pairs_per_step": kept_pairs,
                        "kept_fraction": round(kept_pairs / (wl.N * wl.N * wl.nh * wl.B), 4),
                        "l2": "inputs larger than L2 (3 x %.1f MB of Q/K/V per step)" % (wl.N * wl.nh * wl.D * 2 / 1e6),
-                       "parallelism": f"replicas x{world} (independent layer per GPU)"},
+                       "parallelism": f"replicas x{world} (independent layer per GPU)",
+                       "launch": "CUDA graph replay" if args.graph else "eager launches"},
             "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(achieved, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                          "peak_source": f"{src} bf16 burst", "traffic": traffic},
@@ -483,6 +499,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="replay each step as a captured CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -85,52 +85,79 @@ constexpr int kKStep = 16;   // head-dim slice staged per iteration
 constexpr int kPad = 4;      // smem row padding (floats)
 
 // scores[bh, I, J] = scale * max_{i in I, j in J} sum_d qbar[bh,i,d] kbar[bh,j,d]
+// Two shared-memory buffers: the next head-dim slice is read from global
+// memory into registers while the current one is multiplied, and the 8 x 8
+// register tile is updated with paired fp32 FMAs (two columns per
+// instruction; each sum is still one fp32 fma chain over d, as before).
 template <int R>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
              float* __restrict__ scores, int D, int nsb, int nb, float scale) {
-  __shared__ __align__(16) float As[kKStep][kTile + kPad];
-  __shared__ __align__(16) float Bs[kKStep][kTile + kPad];
+  __shared__ __align__(16) float As[2][kKStep][kTile + kPad];
+  __shared__ __align__(16) float Bs[2][kKStep][kTile + kPad];
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const long long bh = blockIdx.z;
   const int row0 = blockIdx.y * kTile, col0 = blockIdx.x * kTile;
   const float* qa = qbar + bh * (long long)nsb * D;
   const float* ka = kbar + bh * (long long)nsb * D;
-  float acc[8][8];
+  float2 acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
 
-  for (int k0 = 0; k0 < D; k0 += kKStep) {
-    // 128 rows x 16 columns = 512 float4 per operand; two per thread.
+  float4 ga[2], gb[2];
+  auto fetch = [&](int k0) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int f = tid + u * 256;
       const int r = f >> 2, c4 = (f & 3) * 4;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-      if (row0 + r < nsb) a = *reinterpret_cast<const float4*>(qa + (long long)(row0 + r) * D + k0 + c4);
-      if (col0 + r < nsb) b = *reinterpret_cast<const float4*>(ka + (long long)(col0 + r) * D + k0 + c4);
-      As[c4 + 0][r] = a.x; As[c4 + 1][r] = a.y; As[c4 + 2][r] = a.z; As[c4 + 3][r] = a.w;
-      Bs[c4 + 0][r] = b.x; Bs[c4 + 1][r] = b.y; Bs[c4 + 2][r] = b.z; Bs[c4 + 3][r] = b.w;
+      ga[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      gb[u] = ga[u];
+      if (row0 + r < nsb) ga[u] = *reinterpret_cast<const float4*>(qa + (long long)(row0 + r) * D + k0 + c4);
+      if (col0 + r < nsb) gb[u] = *reinterpret_cast<const float4*>(ka + (long long)(col0 + r) * D + k0 + c4);
     }
-    __syncthreads();
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int f = tid + u * 256;
+      const int r = f >> 2, c4 = (f & 3) * 4;
+      As[buf][c4 + 0][r] = ga[u].x; As[buf][c4 + 1][r] = ga[u].y;
+      As[buf][c4 + 2][r] = ga[u].z; As[buf][c4 + 3][r] = ga[u].w;
+      Bs[buf][c4 + 0][r] = gb[u].x; Bs[buf][c4 + 1][r] = gb[u].y;
+      Bs[buf][c4 + 2][r] = gb[u].z; Bs[buf][c4 + 3][r] = gb[u].w;
+    }
+  };
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < D; k0 += kKStep) {
+    const bool more = k0 + kKStep < D;
+    if (more) fetch(k0 + kKStep);
 #pragma unroll
     for (int kk = 0; kk < kKStep; ++kk) {
-      float a[8], b[8];
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
-      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w; a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
-      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w; b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 8 + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float2 b[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                           make_float2(b1.z, b1.w)};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const float2 ai = make_float2(a[i], a[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(ai, b[j], acc[i][j]);
+      }
     }
-    __syncthreads();
+    if (more) {
+      stash(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
   }
 
   // r x r max-pool within the 8 x 8 patch; sub-blocks past nsb do not exist.
@@ -145,7 +172,9 @@ score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
 #pragma unroll
         for (int j = 0; j < R; ++j) {
           const int sr = row0 + ty * 8 + gi * R + i, sc = col0 + tx * 8 + gj * R + j;
-          if (sr < nsb && sc < nsb) m = fmaxf(m, acc[gi * R + i][gj * R + j]);
+          const int cc = gj * R + j;
+          const float2 pr = acc[gi * R + i][cc >> 1];
+          if (sr < nsb && sc < nsb) m = fmaxf(m, (cc & 1) ? pr.y : pr.x);
         }
       const int I = (row0 + ty * 8) / R + gi, J = (col0 + tx * 8) / R + gj;
       if (I < nb && J < nb) scores[(bh * nb + I) * (long long)nb + J] = m * scale;

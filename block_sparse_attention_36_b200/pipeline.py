@@ -109,6 +109,23 @@ class DfsLayer:
         self.attend(stream)
         return self.out
 
+    def capture_graph(self, q, k, v, refresh_mask=True, warmup=2):
+        """Record one whole step (prepare + attend) into a CUDA graph over the
+        given, fixed input buffers; replay it with ``graph.replay()``. Warm-up
+        steps run first (eagerly, on a side stream), so one-time set-up such
+        as building the curve index and raising kernel attributes happens
+        outside the capture."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                self.forward(q, k, v, refresh_mask)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(q, k, v, refresh_mask)
+        return graph
+
     def kept_pairs(self):
         """Valid (query, key) token pairs the kept blocks cover (for FLOP counts)."""
         s = self.shape

@@ -171,3 +171,17 @@ def test_schedule_workload_steps(bsa):
         prev_idx = idx.copy()
         rows = _sample_rows(rng, wl.B, wl.nh, s.nb, 6)
         _check_sampled_attention(layer, (qk["q"], qk["k"], v), rows)
+
+
+def test_graph_replay_matches_eager(bsa):
+    """A whole step captured in a CUDA graph gives the eager result."""
+    wl = synth.WORKLOADS["tiny"]
+    qkv = synth.workload_inputs(wl)
+    q, k, v = (qkv[n].cuda() for n in ("q", "k", "v"))
+    layer = _layer(bsa, wl)
+    eager = layer.forward(q, k, v).clone()
+    graph = layer.capture_graph(q, k, v)
+    layer.out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.out, eager)
