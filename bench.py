@@ -37,7 +37,7 @@ if ROOT not in sys.path:
 
 METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
 # fused gather + pooling (1 launch), score, select, attention, scatter; LVSA: 3 gathers, select, attention, scatter
-KERNELS_PER_STEP = {"topk": 5, "threshold": 5, "lvsa": 6}
+KERNELS_PER_STEP = {"topk": 5, "threshold": 5, "global": 5, "lvsa": 6}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per attention launch from one ncu capture
@@ -74,6 +74,7 @@ def load_peaks():
 
 def workload_config(wl, k, cap):
     sel = {"topk": f"top-k {k}/{wl.nb}", "threshold": f"threshold tau={wl.tau} cap {cap}/{wl.nb}",
+           "global": f"global top {k} of {wl.nb}x{wl.nb} pairs per head",
            "lvsa": f"LVSA T_per={wl.lvsa_T_per} C={wl.lvsa_C} step {wl.lvsa_step}"}[wl.mode]
     return (f"{wl.name}: B={wl.B} nh={wl.nh} D={wl.D} grid {wl.T}x{wl.H}x{wl.W} (N={wl.N}) "
             f"{wl.order} order, blk {wl.blk}, sb {wl.sb}, {sel}")
@@ -188,6 +189,9 @@ def make_layer(bsa, wl):
     elif wl.mode == "threshold":
         cap = wl.ratio_count(wl.cap_num)
         layer = bsa.DfsLayer(s, order=wl.order, mode="threshold", cap=cap, tau=wl.tau)
+    elif wl.mode == "global":
+        k = wl.pair_count(wl.keep_num)
+        layer = bsa.DfsLayer(s, order=wl.order, mode="global", k=k, kcap=s.nb)
     else:
         layer = bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
                              lvsa_step=wl.lvsa_step)

@@ -239,6 +239,97 @@ select_lvsa_kernel(int rows, int nb, long long N, int blk, int P, int T, int T_p
   }
 }
 
+// Global selection (VMoBA, abstract, modification 2): per head (one CTA),
+// the K best (query block, key block) pairs of all nb x nb, equal scores to
+// the lower flat index I * nb + J; rows list their kept J ascending.
+// Radix select on order-preserving 32-bit keys (4 passes of 8 bits with a
+// shared-memory histogram) finds the K-th largest key; ties at the cut are
+// taken in flat-index order through a per-row tie count and its prefix sum.
+__global__ void __launch_bounds__(1024)
+select_global_kernel(const float* __restrict__ scores, int nb, int K, int32_t* __restrict__ kv_idx,
+                     int32_t* __restrict__ kv_cnt, int kcap) {
+  extern __shared__ int tie_before[];   // nb + 1 ints
+  __shared__ unsigned hist[256];
+  __shared__ uint32_t sh_prefix, sh_mask;
+  __shared__ int sh_rem;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const long long bh = blockIdx.x;
+  const float* s = scores + bh * (long long)nb * nb;
+  const long long n = (long long)nb * nb;
+  const bool all = (long long)K >= n, none = K <= 0;
+  if (tid == 0) { sh_prefix = 0u; sh_mask = 0u; sh_rem = K; }
+  __syncthreads();
+  if (!all && !none) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int b = tid; b < 256; b += blockDim.x) hist[b] = 0u;
+      __syncthreads();
+      const uint32_t prefix = sh_prefix, mask = sh_mask;
+      for (long long e = tid; e < n; e += blockDim.x) {
+        const uint32_t key = order_key(__ldg(s + e));
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int rem = sh_rem, cum = 0, b = 255;
+        for (; b > 0; --b) {
+          if (cum + (int)hist[b] >= rem) break;
+          cum += (int)hist[b];
+        }
+        sh_prefix = prefix | ((uint32_t)b << shift);
+        sh_mask = mask | (255u << shift);
+        sh_rem = rem - cum;
+      }
+      __syncthreads();
+    }
+  }
+  const uint32_t cut = sh_prefix;              // the K-th largest key
+  const int ties_needed = sh_rem;              // keys == cut to keep, lowest flat index first
+  // ties per row, then their exclusive prefix over rows
+  for (int r = warp; r < nb; r += nwarps) {
+    int c = 0;
+    if (!all && !none)
+      for (int j = lane; j < nb; j += 32) c += order_key(__ldg(s + (long long)r * nb + j)) == cut ? 1 : 0;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) tie_before[r] = c;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int r = 0; r < nb; ++r) {
+      const int c = tie_before[r];
+      tie_before[r] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r = warp; r < nb; r += nwarps) {
+    int base = 0, ties = tie_before[r];
+    int32_t* out = kv_idx + (bh * nb + r) * (long long)kcap;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      bool take = false, eq = false;
+      if (j < nb && !none) {
+        const uint32_t key = order_key(__ldg(s + (long long)r * nb + j));
+        eq = !all && key == cut;
+        take = all || key > cut;
+      }
+      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      if (eq && ties + __popc(eqb & lt) < ties_needed) take = true;
+      ties += __popc(eqb);
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      const int pos = base + __popc(tb & lt);
+      if (take && pos < kcap) out[pos] = j;
+      base += __popc(tb);
+    }
+    if (lane == 0) {
+      if (base > kcap) atomicOr(&g_select_flags, (uint32_t)DFS_FLAG_KCAP_OVERFLOW);
+      kv_cnt[bh * nb + r] = min(base, kcap);
+    }
+  }
+}
+
 }  // namespace
 
 DFS_DEFINE_FLAG_READER(dfs_detail_flags_select, g_select_flags)
@@ -263,6 +354,17 @@ extern "C" int dfs_select_mask(const dfs_shape* shape, const float* scores, cons
   }
   if (!scores) return DFS_ERR_INVALID_ARG;
   if (!dfs::aligned16(scores)) return DFS_ERR_MISALIGNED;
+  if (prm->mode == DFS_SEL_GLOBAL) {
+    if (prm->k < 0 || kcap < (prm->k < d.nb ? prm->k : d.nb)) return DFS_ERR_INVALID_ARG;
+    if ((long long)d.nb * d.nb > (1LL << 31) - 1 || d.BH > 0x7fffffffLL) return DFS_ERR_UNSUPPORTED;
+    const size_t smem = ((size_t)d.nb + 1) * sizeof(int);
+    if (smem > 200 * 1024) return DFS_ERR_UNSUPPORTED;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(select_global_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return DFS_ERR_CUDA;
+    select_global_kernel<<<(unsigned)d.BH, 1024, smem, cs>>>(scores, d.nb, prm->k, kv_idx, kv_cnt, kcap);
+    return dfs::launch_status();
+  }
   if (prm->mode == DFS_SEL_TOPK) {
     if (prm->k < 0 || kcap < (prm->k < d.nb ? prm->k : d.nb)) return DFS_ERR_INVALID_ARG;
   } else if (prm->mode == DFS_SEL_THRESHOLD) {

@@ -29,6 +29,7 @@ DFS_ORDER_HILBERT3D = 1
 DFS_SEL_TOPK = 0
 DFS_SEL_THRESHOLD = 1
 DFS_SEL_LVSA = 2
+DFS_SEL_GLOBAL = 3
 DFS_WS_BLOCK_SCORE = 0
 
 DFS_FLAG_WAIT_TIMEOUT = 1
@@ -36,7 +37,7 @@ DFS_FLAG_BAD_KV_INDEX = 2
 DFS_FLAG_KCAP_OVERFLOW = 4
 
 ORDERS = {"raster": DFS_ORDER_RASTER, "hilbert3d": DFS_ORDER_HILBERT3D}
-MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA}
+MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA, "global": DFS_SEL_GLOBAL}
 
 # C entry points declared in include/dfsattn.h.
 EXPORTS = (

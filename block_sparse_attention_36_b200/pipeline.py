@@ -29,7 +29,8 @@ class DfsLayer:
                                         lvsa_step=lvsa_step)
         s = shape
         if kcap is None:
-            kcap = {"topk": max(1, min(k, s.nb)), "threshold": max(1, min(cap, s.nb))}.get(mode, s.nb)
+            kcap = {"topk": max(1, min(k, s.nb)), "threshold": max(1, min(cap, s.nb)),
+                    "global": max(1, min(k, s.nb))}.get(mode, s.nb)
         self.kcap = int(kcap)
         self.scale = float(scale) if scale and scale > 0 else 1.0 / math.sqrt(s.D)
         dev = torch.device(device)

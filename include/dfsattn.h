@@ -63,7 +63,7 @@ typedef struct {
 } dfs_shape;
 
 enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1 };
-enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2 };
+enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2, DFS_SEL_GLOBAL = 3 };
 enum { DFS_WS_BLOCK_SCORE = 0 };
 
 /* Device error word bits (dfs_get_error_flags). */
@@ -87,7 +87,14 @@ enum {
  *                              J is kept for query block I when a frame J
  *                              touches lies in the union of the frame sets of
  *                              the frames I touches. A frame is H*W tokens of
- *                              the raster order.                              */
+ *                              the raster order.
+ *   mode = DFS_SEL_GLOBAL    : VMoBA global selection (abstract, modification
+ *                              2): per head, the k best (query block, key
+ *                              block) pairs over all nb * nb of them (equal
+ *                              scores: lower flat index I * nb + J first);
+ *                              each query block lists its kept key blocks
+ *                              ascending and may keep none. k counts pairs
+ *                              per head here.                                  */
 typedef struct {
   int mode;
   int k;
@@ -176,8 +183,8 @@ int dfs_block_score_noalloc(const dfs_shape *shape, const void *qp, const void *
  * Writes, per row (b, h, I), the kept key-block indices in ascending order
  * to kv_idx[((b*nh + h)*nb + I)*kcap + 0 .. cnt-1] (int32) and cnt to
  * kv_cnt[(b*nh + h)*nb + I]. Slots past cnt are not written. kcap >= 1; for
- * top-k kcap >= min(k, nb) and for threshold kcap >= min(cap, nb) are
- * checked on the host; a longer list is truncated to kcap and sets
+ * top-k and global kcap >= min(k, nb) and for threshold kcap >= min(cap,
+ * nb) are checked on the host; a longer list is truncated to kcap and sets
  * DFS_FLAG_KCAP_OVERFLOW.                                                  */
 int dfs_select_mask(const dfs_shape *shape, const float *scores, const dfs_select_params *params,
                     int32_t *kv_idx, int32_t *kv_cnt, int kcap, dfs_stream_t stream);

@@ -6,9 +6,15 @@ Follows
     blocks each query block keeps (top-k of the block importance);
   * VMoBA: Mixture of Block Attention for Video Diffusion Models, abstract,
     modification (3): threshold-based selection keeps as many blocks as their
-    cumulative similarity requires.
+    cumulative similarity requires;
+  * VMoBA, abstract, modification (2): global block selection ranks
+    query-key block pairs across the whole head.
 
 Readings:
+  * global selection keeps, per head, the K highest-scoring (query block, key
+    block) pairs over all nb x nb pairs, equal scores going to the lower flat
+    index I * nb + J; each query block's kept key blocks are listed in
+    ascending order (a query block may keep none); K = ceil(ratio * nb^2);
   * top-k keeps the k largest scores of the row; equal scores go to the lower
     key-block index; no block is forced in (no diagonal or sink block);
   * threshold: p = softmax over the row of the block scores (temperature 1,
@@ -87,6 +93,26 @@ def select(scores, mode, k=0, tau=0.0, cap=0, kcap=None):
                 idx[b, h, I, :kept.size] = kept
                 cnt[b, h, I] = kept.size
     return idx, cnt
+
+
+def global_topk_head(scores_head, K):
+    """Boolean [nb, nb] mask of the K best pairs of one head (ties: lower flat index)."""
+    s = np.asarray(scores_head, dtype=np.float32)
+    nbq, nbk = s.shape
+    flat = s.reshape(-1)
+    K = max(0, min(int(K), flat.size))
+    order = np.lexsort((np.arange(flat.size), -flat.astype(np.float64)))
+    m = np.zeros(flat.size, dtype=bool)
+    m[order[:K]] = True
+    return m.reshape(nbq, nbk)
+
+
+def select_global(scores, K, kcap=None):
+    """Per-head global selection of [B, nh, nb, nb] scores -> (kv_idx, kv_cnt)."""
+    s32 = np.asarray(scores, dtype=np.float32)
+    B, nh = s32.shape[:2]
+    mask = np.stack([np.stack([global_topk_head(s32[b, h], K) for h in range(nh)]) for b in range(B)])
+    return mask_to_lists(mask, kcap)
 
 
 def lists_to_mask(kv_idx, kv_cnt, nbk):

@@ -185,7 +185,7 @@ class Workload:
     blk: int
     sb: int
     order: str            # "hilbert3d" or "raster"
-    mode: str             # "topk", "threshold", "lvsa", "schedule"
+    mode: str             # "topk", "threshold", "lvsa", "schedule", "global"
     keep_num: int = 0     # keep ratio numerator / 100 (top-k)
     tau: float = 0.0
     cap_num: int = 0      # cap ratio numerator / 100 (threshold)
@@ -211,6 +211,10 @@ class Workload:
         """ceil(num/100 * nb) in exact integer arithmetic."""
         return -(-(num * self.nb) // 100)
 
+    def pair_count(self, num: int) -> int:
+        """ceil(num/100 * nb^2): block pairs kept per head by global selection."""
+        return -(-(num * self.nb * self.nb) // 100)
+
 
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 2, 64, 8, 16, 16, 64, 16, "hilbert3d", "topk", keep_num=25),
@@ -219,6 +223,8 @@ WORKLOADS = {
                                 n_steps=50, refresh=5),
     "lvsa_long_video": Workload("lvsa_long_video", 1, 12, 128, 63, 30, 52, 128, 32, "raster", "lvsa",
                                 lvsa_T_per=8, lvsa_C=21, lvsa_step=0),
+    "wan_1p3b_global": Workload("wan_1p3b_global", 1, 12, 128, 21, 30, 52, 128, 32, "hilbert3d", "global",
+                                keep_num=15),
     "hunyuan_layer": Workload("hunyuan_layer", 1, 24, 128, 33, 45, 80, 128, 32, "hilbert3d", "threshold",
                               tau=0.9, cap_num=20),
 }

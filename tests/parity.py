@@ -71,3 +71,28 @@ def assert_attn_close(got, ref, what=""):
     mx, rel = attn_errors(got, ref)
     assert mx <= ATOL_MAX and rel <= RTOL_FRO, f"{what}: max abs {mx:.3e}, rel fro {rel:.3e}"
     return mx, rel
+
+
+def compare_global_masks(g_idx, g_cnt, o_idx, o_cnt, o_scores, K, eps=EPS):
+    """Global selection: per head the kept pair sets must match except pairs
+    whose fp64 oracle score lies within eps of the head's cut-off score (the
+    K-th best), which are excused and counted."""
+    from oracle import selection as sel
+    nb = o_scores.shape[-1]
+    gm = sel.lists_to_mask(np.asarray(g_idx), np.asarray(g_cnt), nb)
+    om = sel.lists_to_mask(np.asarray(o_idx), np.asarray(o_cnt), nb)
+    s64 = np.asarray(o_scores, dtype=np.float64)
+    out = {"bad_rows": 0, "excused_entries": 0, "heads": gm.shape[0] * gm.shape[1], "bad_examples": []}
+    for b in range(gm.shape[0]):
+        for h in range(gm.shape[1]):
+            diff = gm[b, h] ^ om[b, h]
+            if not diff.any():
+                continue
+            cut = s64[b, h][om[b, h]].min() if om[b, h].any() else np.inf
+            bad = diff & (np.abs(s64[b, h] - cut) > eps)
+            if gm[b, h].sum() == om[b, h].sum() and not bad.any():
+                out["excused_entries"] += int(diff.sum())
+            else:
+                out["bad_rows"] += int(bad.any(axis=1).sum())
+                out["bad_examples"].append((b, h, int(diff.sum())))
+    return out

@@ -1,10 +1,11 @@
 """GPU key-block selection against the oracle.
 
 Pages: DFSAttn, Methodology item 3 (top-k budget); VMoBA abstract,
-modification (3) (cumulative-mass threshold); LVSA section 2 (frame mask).
-Given the same fp32 scores, top-k lists are bit-exact (ties included); a
-threshold row may differ only where the oracle's cumulative mass at the
-cut lies within 1e-5 of tau (counted); LVSA lists are bit-exact."""
+modifications (2) (global selection) and (3) (cumulative-mass threshold);
+LVSA section 2 (frame mask). Given the same fp32 scores, top-k and global
+lists are bit-exact (ties included); a threshold row may differ only where
+the oracle's cumulative mass at the cut lies within 1e-5 of tau (counted);
+LVSA lists are bit-exact."""
 import numpy as np
 import pytest
 import torch
@@ -100,3 +101,16 @@ def test_kcap_overflow_is_flagged(lib):
     gi, gc = _select(lib, None, shape, lib.select_params("lvsa", lvsa_T_per=8, lvsa_C=21, lvsa_step=0), 16)
     assert (gc <= 16).all()
     assert lib.dfs_get_error_flags(clear=True) & lib.DFS_FLAG_KCAP_OVERFLOW
+
+
+@pytest.mark.parametrize("nb,K", [(32, 100), (256, 9831), (57, 1), (40, 1600), (40, 0), (300, 4500), (929, 172609)])
+def test_global_selection_bit_exact(lib, nb, K):
+    rng = np.random.default_rng(nb + K)
+    s = (rng.standard_normal((1, 2, nb, nb)) * 2).astype(np.float32)
+    s[0, 1] = np.round(s[0, 1])                           # heavy ties across the head
+    shape = _shape_for(lib, nb)
+    kcap = nb
+    gi, gc = _select(lib, s, shape, lib.select_params("global", k=K), kcap)
+    oi, oc = selection.select_global(s, K, kcap=kcap)
+    _lists_equal(gi, gc, oi, oc)
+    assert gc.reshape(2, -1).sum(axis=1).tolist() == [min(K, nb * nb)] * 2

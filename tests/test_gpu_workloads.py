@@ -19,7 +19,7 @@ import torch
 
 import synth
 from oracle import attention, hilbert, lvsa, pipeline, schedule, scoring, selection
-from tests.parity import assert_attn_close, compare_masks
+from tests.parity import assert_attn_close, compare_global_masks, compare_masks
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +40,9 @@ def _layer(bsa, wl, **kw):
     if wl.mode == "lvsa":
         return bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
                             lvsa_step=wl.lvsa_step, want_lse=True, **kw)
+    if wl.mode == "global":
+        return bsa.DfsLayer(s, order=wl.order, mode="global", k=wl.pair_count(wl.keep_num), kcap=s.nb,
+                            want_lse=True, **kw)
     raise ValueError(wl.mode)
 
 
@@ -105,7 +108,7 @@ def test_tiny_workload_end_to_end(bsa):
     assert_attn_close(out, hilbert.unpermute_tokens(full, res["perm"]), "tiny output, GPU lists")
 
 
-@pytest.mark.parametrize("name", ["wan_1p3b_layer", "hunyuan_layer", "lvsa_long_video"])
+@pytest.mark.parametrize("name", ["wan_1p3b_layer", "hunyuan_layer", "lvsa_long_video", "wan_1p3b_global"])
 def test_full_size_workload(bsa, name):
     wl = synth.WORKLOADS[name]
     qkv = synth.workload_inputs(wl)
@@ -129,6 +132,10 @@ def test_full_size_workload(bsa, name):
         if wl.mode == "topk":
             oi, oc = selection.select(ref_scores, "topk", k=wl.ratio_count(wl.keep_num), kcap=layer.kcap)
             cmp = compare_masks(layer.kv_idx.cpu().numpy(), layer.kv_cnt.cpu().numpy(), oi, oc, ref_scores, "topk")
+        elif wl.mode == "global":
+            K = wl.pair_count(wl.keep_num)
+            oi, oc = selection.select_global(ref_scores, K, kcap=layer.kcap)
+            cmp = compare_global_masks(layer.kv_idx.cpu().numpy(), layer.kv_cnt.cpu().numpy(), oi, oc, ref_scores, K)
         else:
             cap = wl.ratio_count(wl.cap_num)
             oi, oc = selection.select(ref_scores, "threshold", tau=wl.tau, cap=cap, kcap=layer.kcap)

@@ -90,3 +90,29 @@ def test_select_lists_and_mask_roundtrip():
     assert (m.sum(-1) == 3).all()
     idx2, cnt2 = selection.mask_to_lists(m, 4)
     assert np.array_equal(idx, idx2) and np.array_equal(cnt, cnt2)
+
+
+def test_global_selection_rank_count_brute_force():
+    # pair (I, J) kept iff fewer than K pairs outrank it (higher score, or
+    # equal score and lower flat index)
+    rng = np.random.default_rng(7)
+    for trial in range(60):
+        nb = int(rng.integers(1, 7))
+        s = rng.integers(-2, 3, size=(nb, nb)).astype(np.float32)
+        K = int(rng.integers(0, nb * nb + 1))
+        m = selection.global_topk_head(s, K)
+        flat = s.reshape(-1)
+        for f in range(nb * nb):
+            better = sum(1 for g in range(nb * nb) if flat[g] > flat[f] or (flat[g] == flat[f] and g < f))
+            assert m.reshape(-1)[f] == (better < K)
+        assert m.sum() == K
+
+
+def test_global_selection_lists():
+    s = np.zeros((1, 1, 3, 3), dtype=np.float32)
+    s[0, 0, 2, 0] = 5.0
+    s[0, 0, 0, 2] = 4.0
+    idx, cnt = selection.select_global(s, 3)
+    # best two pairs, then the lowest flat index among the zero ties: (0, 0)
+    assert list(cnt[0, 0]) == [2, 0, 1]
+    assert list(idx[0, 0, 0, :2]) == [0, 2] and idx[0, 0, 2, 0] == 0
