@@ -116,14 +116,40 @@ __device__ void hilbert_cell(Box cur, long long r, int out[3]) {
   out[0] = cur.p[0]; out[1] = cur.p[1]; out[2] = cur.p[2];
 }
 
-__global__ void hilbert_index_kernel(int T, int H, int W, int order, int32_t* __restrict__ perm,
-                                     int32_t* __restrict__ inv) {
+// Cell of rank i in tile-major order (tiles of ct x ch x cw in raster order,
+// clipped at the far edges; raster order inside a tile). Every time slab of
+// tiles before the last is full, every row of tiles before the last in a
+// slab is full, and so on, so each level is one division.
+__device__ __forceinline__ long long tiled_cell(long long i, int T, int H, int W, int ct, int ch, int cw) {
+  const long long slab = (long long)ct * H * W;
+  const long long a = i / slab;
+  long long r = i - a * slab;
+  const int tt = min(ct, T - (int)a * ct);
+  const long long row = (long long)tt * ch * W;
+  const long long b = r / row;
+  r -= b * row;
+  const int hh = min(ch, H - (int)b * ch);
+  const long long cube = (long long)tt * hh * cw;
+  const long long c = r / cube;
+  r -= c * cube;
+  const int ww = min(cw, W - (int)c * cw);
+  const long long t = a * ct + r / ((long long)hh * ww);
+  const long long h = b * ch + (r / ww) % hh;
+  const long long w = c * cw + r % ww;
+  return (t * H + h) * W + w;
+}
+
+__global__ void hilbert_index_kernel(int T, int H, int W, int order, int ct, int ch, int cw,
+                                     int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   const long long N = (long long)T * H * W;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= N) return;
   long long n;
   if (order == DFS_ORDER_RASTER) {
     n = i;
+  } else if (order == DFS_ORDER_TILE2D || order == DFS_ORDER_TILE3D) {
+    n = tiled_cell(i, T, H, W, ct, ch, cw);
+    if (n < 0 || n >= N) n = 0;  // unreachable for valid shapes; keeps the write in bounds
   } else {
     // Major axis: the longest side, ties to W, then H, then T; the other two
     // in the order W, H, T.
@@ -268,6 +294,18 @@ gather_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, con
   }
 }
 
+bool valid_order(int order) {
+  return order == DFS_ORDER_RASTER || order == DFS_ORDER_HILBERT3D || order == DFS_ORDER_TILE2D ||
+         order == DFS_ORDER_TILE3D;
+}
+
+// Tile extents of the tiled orders (blk tokens per full tile).
+void tile_dims(int order, int blk, int* ct, int* ch, int* cw) {
+  if (order == DFS_ORDER_TILE2D) { *ct = 1; *ch = 8; *cw = blk / 8; }
+  else if (order == DFS_ORDER_TILE3D) { *ct = 2; *ch = 8; *cw = blk / 16; }
+  else { *ct = *ch = *cw = 1; }
+}
+
 }  // namespace
 
 DFS_DEFINE_FLAG_READER(dfs_detail_flags_perm, g_perm_flags)
@@ -278,7 +316,7 @@ extern "C" int dfs_hilbert_perm(const dfs_shape* shape, int order, int32_t* perm
   dfs::Dims d;
   int st = dfs::check_shape(shape, &d, false);
   if (st != DFS_OK) return st;
-  if (order != DFS_ORDER_RASTER && order != DFS_ORDER_HILBERT3D) return DFS_ERR_INVALID_ARG;
+  if (!valid_order(order)) return DFS_ERR_INVALID_ARG;
   if (!perm || (build_index && !inv)) return DFS_ERR_INVALID_ARG;
   const void* srcs[3] = {q, k, v};
   void* dsts[3] = {qp, kp, vp};
@@ -290,7 +328,9 @@ extern "C" int dfs_hilbert_perm(const dfs_shape* shape, int order, int32_t* perm
   if (build_index) {
     const int threads = 256;
     const long long grid = (d.N + threads - 1) / threads;
-    hilbert_index_kernel<<<(unsigned)grid, threads, 0, cs>>>(d.T, d.H, d.W, order, perm, inv);
+    int ct = 1, ch = 1, cw = 1;
+    tile_dims(order, d.blk, &ct, &ch, &cw);
+    hilbert_index_kernel<<<(unsigned)grid, threads, 0, cs>>>(d.T, d.H, d.W, order, ct, ch, cw, perm, inv);
     st = dfs::launch_status();
     if (st != DFS_OK) return st;
   }
@@ -318,7 +358,7 @@ extern "C" int dfs_hilbert_perm_pooled(const dfs_shape* shape, int order, int32_
   dfs::Dims d;
   int st = dfs::check_shape(shape, &d, true);
   if (st != DFS_OK) return st;
-  if (order != DFS_ORDER_RASTER && order != DFS_ORDER_HILBERT3D) return DFS_ERR_INVALID_ARG;
+  if (!valid_order(order)) return DFS_ERR_INVALID_ARG;
   if (!perm || (build_index && !inv)) return DFS_ERR_INVALID_ARG;
   if (!q || !k || !qp || !kp) return DFS_ERR_INVALID_ARG;
   if ((v == nullptr) != (vp == nullptr)) return DFS_ERR_INVALID_ARG;
@@ -334,7 +374,9 @@ extern "C" int dfs_hilbert_perm_pooled(const dfs_shape* shape, int order, int32_
   if (build_index) {
     const int threads = 256;
     const long long grid = (d.N + threads - 1) / threads;
-    hilbert_index_kernel<<<(unsigned)grid, threads, 0, cs>>>(d.T, d.H, d.W, order, perm, inv);
+    int ct = 1, ch = 1, cw = 1;
+    tile_dims(order, d.blk, &ct, &ch, &cw);
+    hilbert_index_kernel<<<(unsigned)grid, threads, 0, cs>>>(d.T, d.H, d.W, order, ct, ch, cw, perm, inv);
     st = dfs::launch_status();
     if (st != DFS_OK) return st;
   }

@@ -36,7 +36,10 @@ DFS_FLAG_WAIT_TIMEOUT = 1
 DFS_FLAG_BAD_KV_INDEX = 2
 DFS_FLAG_KCAP_OVERFLOW = 4
 
-ORDERS = {"raster": DFS_ORDER_RASTER, "hilbert3d": DFS_ORDER_HILBERT3D}
+DFS_ORDER_TILE2D = 2
+DFS_ORDER_TILE3D = 3
+ORDERS = {"raster": DFS_ORDER_RASTER, "hilbert3d": DFS_ORDER_HILBERT3D, "tile2d": DFS_ORDER_TILE2D,
+          "tile3d": DFS_ORDER_TILE3D}
 MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA, "global": DFS_SEL_GLOBAL}
 
 # C entry points declared in include/dfsattn.h.

@@ -62,7 +62,7 @@ typedef struct {
   int blk, sb;
 } dfs_shape;
 
-enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1 };
+enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1, DFS_ORDER_TILE2D = 2, DFS_ORDER_TILE3D = 3 };
 enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2, DFS_SEL_GLOBAL = 3 };
 enum { DFS_WS_BLOCK_SCORE = 0 };
 
@@ -108,7 +108,12 @@ typedef struct {
  * If build_index != 0, first writes perm[N] and inv[N] (int32, device) for
  * `order`: DFS_ORDER_HILBERT3D is the generalised 3D Hilbert curve over the
  * whole T x H x W box (recursive box splitting; starts at (0,0,0), its major
- * axis is the longest side, ties W, H, T); DFS_ORDER_RASTER is the identity.
+ * axis is the longest side, ties W, H, T); DFS_ORDER_RASTER is the identity;
+ * DFS_ORDER_TILE2D / DFS_ORDER_TILE3D are the 2-D / 3-D block partitions of
+ * "VMoBA: Mixture of Block Attention for Video Diffusion Models" (abstract,
+ * modification 1), read as tile-major orders: tiles of 1 x 8 x (blk/8)
+ * tokens (one frame) or 2 x 8 x (blk/16) tokens, in raster order over the
+ * tile grid, clipped at its far edges, raster order inside each tile.
  * The index depends only on (T, H, W, order): callers build it once and
  * reuse it with build_index = 0.
  * Then gathers each non-NULL input x in {q, k, v}, bf16 [B, N, nh, D]

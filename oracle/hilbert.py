@@ -164,11 +164,50 @@ def raster_perm(T, H, W):
     return perm, perm.copy()
 
 
-def make_perm(order, T, H, W):
+def tile_dims(order, blk):
+    """Tile (t, h, w) extents of the tiled orders: blk tokens per full tile.
+
+    Reading of VMoBA: Mixture of Block Attention for Video Diffusion Models,
+    abstract, modification (1) (1-D, 2-D and 3-D block partitions; the
+    abstract gives no tile shapes): 2-D tiles are 1 x 8 x (blk/8) patches of
+    one frame, 3-D tiles are 2 x 8 x (blk/16) cubes; 1-D is the raster order.
+    """
+    if order == "tile2d":
+        return (1, 8, blk // 8)
+    if order == "tile3d":
+        return (2, 8, blk // 16)
+    raise ValueError(order)
+
+
+def tiled_cells(T, H, W, tile):
+    """Cells in tile-major order: tiles in raster order over the tile grid
+    (tiles clipped at the grid's far edges), raster order inside a tile."""
+    ct, ch, cw = tile
+    out = []
+    for t0 in range(0, T, ct):
+        for h0 in range(0, H, ch):
+            for w0 in range(0, W, cw):
+                for t in range(t0, min(t0 + ct, T)):
+                    for h in range(h0, min(h0 + ch, H)):
+                        for w in range(w0, min(w0 + cw, W)):
+                            out.append((t, h, w))
+    return out
+
+
+def tiled_perm(T, H, W, tile):
+    perm = raster_index(tiled_cells(T, H, W, tile), H, W).astype(np.int32)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=np.int32)
+    return perm, inv
+
+
+def make_perm(order, T, H, W, blk=128):
     if order == "hilbert3d":
         return hilbert_perm(T, H, W)
     if order == "raster":
         return raster_perm(T, H, W)
+    if order in ("tile2d", "tile3d"):
+        return tiled_perm(T, H, W, tile_dims(order, blk))
     raise ValueError(order)
 
 

@@ -34,7 +34,7 @@ def run(q, k, v, *, T, H, W, blk, sb, order, mode, k_keep=0, tau=0.0, cap=0,
     B, N, nh, D = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    perm, inv = hilbert.make_perm(order, T, H, W)
+    perm, inv = hilbert.make_perm(order, T, H, W, blk)
     qp, kp, vp = (hilbert.permute_tokens(x, perm) for x in (q, k, v))
     nb = -(-N // blk)
     res = {"perm": perm, "inv": inv, "qp": qp, "kp": kp, "vp": vp}

@@ -92,3 +92,19 @@ def test_partial_tensors(lib):
     operm, _ = hilbert.hilbert_perm(T, H, W)
     assert np.array_equal(kp.cpu().view(torch.int16).numpy(),
                           hilbert.permute_tokens(k.cpu().view(torch.int16).numpy(), operm))
+
+
+@pytest.mark.parametrize("order", ["tile2d", "tile3d"])
+@pytest.mark.parametrize("grid,blk", [((8, 16, 16), 64), ((21, 30, 52), 128), ((3, 5, 7), 64), ((63, 30, 52), 128),
+                                      ((33, 45, 80), 128), ((1, 1, 100), 128), ((5, 17, 9), 128)])
+def test_tiled_orders_match_oracle(lib, order, grid, blk):
+    T, H, W = grid
+    N = T * H * W
+    perm = torch.empty(N, dtype=torch.int32, device="cuda")
+    inv = torch.empty(N, dtype=torch.int32, device="cuda")
+    s = lib.Shape(1, 1, 64, T, H, W, blk, 16)
+    lib.dfs_hilbert_perm(s, order, perm, inv, 1, None, None, None, None, None, None)
+    torch.cuda.synchronize()
+    operm, oinv = hilbert.make_perm(order, T, H, W, blk)
+    assert np.array_equal(perm.cpu().numpy(), operm)
+    assert np.array_equal(inv.cpu().numpy(), oinv)

@@ -99,3 +99,28 @@ def test_pipeline_tiny_grid_full_keep_is_dense():
                        mode="topk", k_keep=4)
     dense = attention.dense_attention(*(np.transpose(x, (0, 2, 1, 3)) for x in (q, k, v)))
     assert np.abs(res["out"] - np.transpose(dense, (0, 2, 1, 3))).max() < 1e-12
+
+
+def test_recall_closed_forms():
+    from oracle import recall
+    rng = np.random.default_rng(9)
+    T, H, W, nh, D, blk = 2, 4, 4, 1, 4, 8
+    N = T * H * W
+    q = rng.standard_normal((1, N, nh, D))
+    k = rng.standard_normal((1, N, nh, D))
+    perm, _ = hilbert.make_perm("hilbert3d", T, H, W)
+    nb = N // blk
+    full = np.tile(np.arange(nb, dtype=np.int32), (1, 1, nb, 1))
+    cnt = np.full((1, 1, nb), nb, dtype=np.int32)
+    qs = [(0, 0, n) for n in range(N)]
+    assert abs(recall.recall(q, k, perm, full, cnt, blk, qs) - 1.0) < 1e-12     # everything kept
+    none = np.zeros((1, 1, nb), dtype=np.int32)
+    assert recall.recall(q, k, perm, full, none, blk, qs) == 0.0               # nothing kept
+    # one block kept: the mass of that block's keys, by brute force
+    one = np.zeros((1, 1, nb, 1), dtype=np.int32)
+    ones = np.ones((1, 1, nb), dtype=np.int32)
+    n = 5
+    s = [sum(q[0, n, 0, d] * k[0, m, 0, d] for d in range(D)) / 2.0 for m in range(N)]
+    e = np.exp(np.array(s) - max(s))
+    ref = e[perm[:blk]].sum() / e.sum()
+    assert abs(recall.recall(q, k, perm, one, ones, blk, [(0, 0, n)]) - ref) < 1e-12

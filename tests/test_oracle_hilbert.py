@@ -142,3 +142,32 @@ def test_permute_roundtrip():
     for i in range(T * H * W):
         assert np.array_equal(xp[0, :, i, :], x[0, perm[i], :, :])
     assert np.array_equal(hilbert.unpermute_tokens(xp, perm), x)
+
+
+@pytest.mark.parametrize("order", ["tile2d", "tile3d"])
+@pytest.mark.parametrize("T,H,W,blk", [(8, 16, 16, 64), (21, 30, 52, 128), (4, 16, 32, 128), (3, 5, 7, 64)])
+def test_tiled_orders(order, T, H, W, blk):
+    perm, inv = hilbert.make_perm(order, T, H, W, blk)
+    N = T * H * W
+    assert np.array_equal(np.sort(perm), np.arange(N)) and np.array_equal(inv[perm], np.arange(N))
+    ct, ch, cw = hilbert.tile_dims(order, blk)
+    assert ct * ch * cw == blk
+    t, r = np.divmod(perm, H * W)
+    h, w = np.divmod(r, W)
+    # every tile is one contiguous run of the order (tile id from integer division)
+    tid = ((t // ct) * (-(-H // ch)) + h // ch) * (-(-W // cw)) + w // cw
+    assert 1 + np.count_nonzero(np.diff(tid)) == len(np.unique(tid))
+    assert np.all(np.diff(tid) >= 0)                     # tiles in raster order
+    if T % ct == 0 and H % ch == 0 and W % cw == 0:
+        # then every block of blk consecutive tokens is exactly one full tile
+        for b0 in range(0, N, blk):
+            sl = slice(b0, b0 + blk)
+            assert (t[sl].max() - t[sl].min() + 1, h[sl].max() - h[sl].min() + 1,
+                    w[sl].max() - w[sl].min() + 1) == (ct, ch, cw)
+
+
+def test_tile2d_first_block_by_hand():
+    # 1 x 16 x 32 grid, blk 128: the first block is rows 0-7, columns 0-15
+    perm, _ = hilbert.make_perm("tile2d", 1, 16, 32, 128)
+    assert list(perm[:18]) == list(range(16)) + [32, 33]
+    assert perm[127] == 7 * 32 + 15 and perm[128] == 16
