@@ -194,7 +194,7 @@ def make_layer(bsa, wl):
         layer = bsa.DfsLayer(s, order=wl.order, mode="global", k=k, kcap=s.nb)
     else:
         layer = bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
-                             lvsa_step=wl.lvsa_step)
+                             lvsa_step=wl.lvsa_step, frame_exact=wl.frame_exact)
     return layer, k, cap
 
 
@@ -441,6 +441,11 @@ def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, steps=1):
             t_mask = t_mask / (h + 1) * wl.nh
             break
     heads_done = len(per_head)
+    allowed = None
+    if wl.frame_exact:
+        fa = lvsa.frame_allowed(wl.T, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step)
+        P = wl.H * wl.W
+        allowed = lambda qs, ks: fa[np.asarray(qs)[:, None] // P, np.asarray(ks)[None, :] // P]
     deadline = time.perf_counter() + max(1.0, budget_s - (time.perf_counter() - t0))
     rows_total = wl.nb * wl.nh * wl.B
     while time.perf_counter() < deadline:
@@ -448,7 +453,7 @@ def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, steps=1):
         I = int(rng.integers(0, wl.nb))
         qp, kp, vp, idx, cnt = per_head[h]
         t1 = time.perf_counter()
-        attention.block_sparse_attention(qp, kp, vp, idx, cnt, wl.blk, rows=[(0, 0, I)])
+        attention.block_sparse_attention(qp, kp, vp, idx, cnt, wl.blk, rows=[(0, 0, I)], allowed=allowed)
         t_attn += time.perf_counter() - t1
         n_rows += 1
         rows_q = min(wl.blk, wl.N - I * wl.blk)

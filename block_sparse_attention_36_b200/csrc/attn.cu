@@ -37,6 +37,7 @@
 
 #include "common.cuh"
 #include "exp2_poly.cuh"
+#include "lvsa.cuh"
 #include "sm100_ptx.cuh"
 
 // Every DFS_ATTN_EXP2_EMU-th pair of softmax exponentials is computed on the
@@ -105,12 +106,24 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
     mma_ts_warp(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <int D, int BLK, int EMU>
+// Frame-exact LVSA masking inside the kept blocks (raster token order, P
+// tokens per frame, P >= BLK so a block touches at most two frames and the
+// 2 * BLK query rows of a CTA at most three). The CTA first tabulates, for
+// each of its query frames, the bit set A(t) over all T key frames in
+// shared memory; the softmax then masks by two bit lookups per key block.
+struct FrameMask {
+  int P, T, T_per, s0, C, nG;
+};
+constexpr int kFrameRows = 3;
+constexpr int kMaxFrames = 4096;
+__host__ __device__ constexpr int frame_words(int T) { return (T + 31) / 32; }
+
+template <int D, int BLK, int EMU, bool FRAME>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ kv_idx,
                 const int32_t* __restrict__ kv_cnt, int kcap, int N, int nb, float scale_log2,
-                __nv_bfloat16* __restrict__ op, float* __restrict__ lse, int max_list) {
+                __nv_bfloat16* __restrict__ op, float* __restrict__ lse, int max_list, FrameMask fm) {
   using C = Cfg<D, BLK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -164,6 +177,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0) bars->n_kv[x] = base;
   }
   if (warp == 1) tmem_alloc(&bars->tmem_base, C::kTmemCols);
+  uint32_t* ftab = reinterpret_cast<uint32_t*>(lists + 2 * max_list);
+  const int qf_lo = FRAME ? (I0 * BLK) / fm.P : 0;
+  if (FRAME && warp >= 4) {
+    const int words = frame_words(fm.T);
+    for (int w = threadIdx.x - 128; w < kFrameRows * words; w += kThreads - 128) {
+      const int t = min(fm.T - 1, qf_lo + w / words);
+      const int f_base = (w % words) * 32;
+      uint32_t bits = 0;
+      for (int b = 0; b < 32 && f_base + b < fm.T; ++b)
+        if (dfs::lvsa_in_frame_set(f_base + b, t, fm.T, fm.T_per, fm.s0, fm.C, fm.nG)) bits |= 1u << b;
+      ftab[w] = bits;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -293,6 +319,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float m = -INFINITY;                            // running max (log2 units)
     float l = 0.f;                                  // running row sum
     bool ok = true;
+    const uint32_t* frow = ftab;                    // A(query frame) as bits
+    if (FRAME) frow += (min(fm.T - 1, (I * BLK + r) / fm.P) - qf_lo) * frame_words(fm.T);
     for (int j = 0; j < nx; ++j) {
       if (!mbar_wait_bounded(&bars->s_full[x], (uint32_t)(j & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       tc_fence_after();
@@ -309,6 +337,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int e = 0; e < BLK; ++e)
           if (e >= rem) sv[e] = -INFINITY;
+      }
+      if (FRAME) {
+        // Keys of this block lie in frames f0 (columns < cb) and f0 + 1;
+        // drop the frame(s) outside A(query frame).
+        const int k0 = list[j] * BLK;
+        const int f0 = k0 / fm.P;
+        const int cb = min(BLK, (f0 + 1) * fm.P - k0);
+        const bool a0 = (frow[f0 >> 5] >> (f0 & 31)) & 1u;
+        const bool a1 = cb >= BLK || (f0 + 1 < fm.T && ((frow[(f0 + 1) >> 5] >> ((f0 + 1) & 31)) & 1u));
+        if (!a0 || !a1) {
+#pragma unroll
+          for (int e = 0; e < BLK; ++e)
+            if (e < cb ? !a0 : !a1) sv[e] = -INFINITY;
+        }
       }
       // row maximum: eight independent chains of three-input maxima
       float mx8[8];
@@ -334,7 +376,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       // P = 2^(s * scale_log2 - m), bf16, written over S_X (fully read).
       const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_use, -m_use);
+      // A row whose keys so far are all masked has no maximum yet: its
+      // exponentials are all 2^-inf = 0 whatever is subtracted.
+      const float m_sub = (FRAME && m_use == -INFINITY) ? 0.f : m_use;
+      const float2 nm2 = make_float2(-m_sub, -m_sub);
       float2 acc[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
@@ -361,7 +406,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // O_X may be rescaled here: s_full(j) was committed after PV_X(j-1)
       // by the same thread, so PV_X(j-1) has completed.
       if (rescale) {
-        const float alpha = ex2(m - m_use);
+        // (a row with no unmasked key yet has O = 0 and l = 0)
+        const float alpha = (FRAME && m == -INFINITY) ? 0.f : ex2(m - m_use);
         const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -457,9 +503,10 @@ bool make_map(CUtensorMap* map, const void* base, long long N, int D, long long 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK, int EMU>
+template <int D, int BLK, int EMU, bool FRAME>
 int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
-                const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t st) {
+                const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t st,
+                FrameMask fm) {
   using C = Cfg<D, BLK>;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qp, d.N, D, d.BH, kQRows) || !make_map(&mk, kp, d.N, D, d.BH, BLK) ||
@@ -467,19 +514,20 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
     return DFS_ERR_CUDA;
   const int max_list = min(kcap, d.nb);
   size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + 2 * (size_t)max_list * sizeof(int32_t);
+  if (FRAME) smem += (size_t)kFrameRows * frame_words(fm.T) * sizeof(uint32_t);
   if (smem > 232448) return DFS_ERR_UNSUPPORTED;
   // Tensor memory per SM is 512 columns: a 512-column CTA must be alone on
   // its SM and a 256-column CTA may share it with one other, so shared
   // memory is padded to make the scheduler place CTAs that way.
   const size_t min_smem = (C::kTmemCols == 512) ? 120 * 1024 : 80 * 1024;
   if (smem < min_smem) smem = min_smem;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, EMU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, EMU, FRAME>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return DFS_ERR_CUDA;
   dim3 grid((unsigned)((d.nb + 1) / 2), (unsigned)d.BH);
   const float scale_log2 = scale * 1.4426950408889634f;
-  attn_fwd_kernel<D, BLK, EMU><<<grid, kThreads, smem, st>>>(mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb,
-                                                             scale_log2, (__nv_bfloat16*)op, lse, max_list);
+  attn_fwd_kernel<D, BLK, EMU, FRAME><<<grid, kThreads, smem, st>>>(
+      mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb, scale_log2, (__nv_bfloat16*)op, lse, max_list, fm);
   return dfs::launch_status();
 }
 
@@ -487,25 +535,63 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
 
 DFS_DEFINE_FLAG_READER(dfs_detail_flags_attn, g_attn_flags)
 
-extern "C" int dfs_sparse_attn_fwd(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
-                                   const int32_t* kv_idx, const int32_t* kv_cnt, int kcap, float scale, void* op,
-                                   float* lse, dfs_stream_t stream) {
-  dfs::Dims d;
-  int st = dfs::check_shape(shape, &d, false);
+namespace {
+
+int check_attn_args(const dfs_shape* shape, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
+                    const int32_t* kv_cnt, int kcap, void* op, float* lse, dfs::Dims* d) {
+  int st = dfs::check_shape(shape, d, false);
   if (st != DFS_OK) return st;
   if (!qp || !kp || !vp || !kv_idx || !kv_cnt || !op || kcap < 1) return DFS_ERR_INVALID_ARG;
   if (!dfs::aligned16(qp) || !dfs::aligned16(kp) || !dfs::aligned16(vp) || !dfs::aligned16(op) ||
       (lse && !dfs::aligned16(lse)))
     return DFS_ERR_MISALIGNED;
-  if (d.N >= (1LL << 31) || d.BH > 65535) return DFS_ERR_UNSUPPORTED;
-  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
-  cudaStream_t cs = (cudaStream_t)stream;
+  if (d->N >= (1LL << 31) || d->BH > 65535) return DFS_ERR_UNSUPPORTED;
+  return DFS_OK;
+}
+
+template <bool FRAME>
+int dispatch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
+                  const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t cs,
+                  FrameMask fm) {
   constexpr int kEmu = DFS_ATTN_EXP2_EMU;
   if (d.D == 128 && d.blk == 128)
-    return launch_attn<128, 128, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+    return launch_attn<128, 128, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
   if (d.D == 128 && d.blk == 64)
-    return launch_attn<128, 64, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+    return launch_attn<128, 64, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
   if (d.D == 64 && d.blk == 128)
-    return launch_attn<64, 128, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
-  return launch_attn<64, 64, kEmu>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs);
+    return launch_attn<64, 128, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
+  return launch_attn<64, 64, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
+}
+
+}  // namespace
+
+extern "C" int dfs_sparse_attn_fwd(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
+                                   const int32_t* kv_idx, const int32_t* kv_cnt, int kcap, float scale, void* op,
+                                   float* lse, dfs_stream_t stream) {
+  dfs::Dims d;
+  const int st = check_attn_args(shape, qp, kp, vp, kv_idx, kv_cnt, kcap, op, lse, &d);
+  if (st != DFS_OK) return st;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
+  return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream,
+                              FrameMask{1, 1, 1, 0, 1, 0});
+}
+
+extern "C" int dfs_sparse_attn_lvsa_fwd(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
+                                        const int32_t* kv_idx, const int32_t* kv_cnt, int kcap, float scale,
+                                        const dfs_select_params* lvsa, void* op, float* lse, dfs_stream_t stream) {
+  dfs::Dims d;
+  const int st = check_attn_args(shape, qp, kp, vp, kv_idx, kv_cnt, kcap, op, lse, &d);
+  if (st != DFS_OK) return st;
+  if (!lvsa || lvsa->lvsa_T_per < 1 || lvsa->lvsa_C < 1 || lvsa->lvsa_step < 0) return DFS_ERR_INVALID_ARG;
+  const long long P = (long long)d.H * d.W;
+  if (P < d.blk || d.T > kMaxFrames) return DFS_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
+  FrameMask fm;
+  fm.P = (int)P;
+  fm.T = d.T;
+  fm.T_per = lvsa->lvsa_T_per;
+  fm.s0 = lvsa->lvsa_step % lvsa->lvsa_T_per;
+  fm.C = lvsa->lvsa_C;
+  fm.nG = (fm.s0 < d.T) ? (d.T - 1 - fm.s0) / fm.T_per + 1 : 0;
+  return dispatch_attn<true>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream, fm);
 }

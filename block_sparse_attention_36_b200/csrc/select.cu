@@ -18,6 +18,7 @@
 // warp-wide mass sums. Kept columns are emitted in ascending order with
 // ballots and popcounts; equal keys at the cut go to the lowest columns.
 #include "common.cuh"
+#include "lvsa.cuh"
 
 namespace {
 
@@ -178,33 +179,6 @@ select_scores_kernel(const float* __restrict__ scores, int rows, int nb, int mod
   }
 }
 
-// Number of anchor frames in [lo, hi] (anchors: f mod T_per == s0).
-__device__ __forceinline__ int anchors_in(int lo, int hi, int T_per, int s0) {
-  if (hi < lo) return 0;
-  // count of f in [lo, hi] with f = s0 + m * T_per, m integer
-  auto fl = [](int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); };
-  return fl(hi - s0, T_per) - fl(lo - 1 - s0, T_per);
-}
-
-// Is frame f in A(t)? Anchors always; otherwise f must be among the
-// (C - |G|) non-anchor frames nearest to t in the scan order
-// t, t-1, t+1, t-2, t+2, ... (frames outside [0, T) skipped).
-__device__ __forceinline__ bool in_frame_set(int f, int t, int T, int T_per, int s0, int C, int nG) {
-  if (((f - s0) % T_per + T_per) % T_per == 0) return true;
-  const int need = C - nG;
-  if (need <= 0) return false;
-  const int dist = f > t ? f - t : t - f;
-  // non-anchor frames scanned before f: all of (t-dist, t+dist) ...
-  int lo = max(0, t - dist + 1), hi = min(T - 1, t + dist - 1);
-  int before = (hi >= lo) ? (hi - lo + 1) - anchors_in(lo, hi, T_per, s0) : 0;
-  // ... plus t - dist when f = t + dist (the earlier side goes first)
-  if (dist > 0 && f > t) {
-    const int g = t - dist;
-    if (g >= 0 && ((g - s0) % T_per + T_per) % T_per != 0) ++before;
-  }
-  return before < need;
-}
-
 __global__ void __launch_bounds__(256)
 select_lvsa_kernel(int rows, int nb, long long N, int blk, int P, int T, int T_per, int C, int s0,
                    int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, int kcap) {
@@ -212,7 +186,7 @@ select_lvsa_kernel(int rows, int nb, long long N, int blk, int P, int T, int T_p
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int I = (int)(row % nb);
-  const int nG = (s0 < T) ? (T - 1 - s0) / T_per + 1 : 0;
+  const int nG = dfs::lvsa_anchor_count(T, T_per, s0);
   const int qf0 = (int)(((long long)I * blk) / P);
   const int qf1 = (int)((min((long long)I * blk + blk, N) - 1) / P);
   int32_t* out = kv_idx + row * (long long)kcap;
@@ -226,7 +200,7 @@ select_lvsa_kernel(int rows, int nb, long long N, int blk, int P, int T, int T_p
       const int kf1 = (int)((min((long long)J * blk + blk, N) - 1) / P);
       for (int f = kf0; f <= kf1 && !take; ++f)
         for (int t = qf0; t <= qf1 && !take; ++t)
-          take = in_frame_set(f, t, T, T_per, s0, C, nG);
+          take = dfs::lvsa_in_frame_set(f, t, T, T_per, s0, C, nG);
     }
     const unsigned tb = __ballot_sync(0xffffffffu, take);
     const int pos = base + __popc(tb & lt);

@@ -46,7 +46,7 @@ MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_L
 EXPORTS = (
     "dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd", "dfs_unperm",
     "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version", "dfs_block_score_noalloc",
-    "dfs_hilbert_perm_pooled", "dfs_block_score_pooled",
+    "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd",
 )
 
 
@@ -72,6 +72,7 @@ def _load():
     lib.dfs_block_score_noalloc.argtypes = [sp, P, P, F, P, P]
     lib.dfs_hilbert_perm_pooled.argtypes = [sp, I, P, P, I, P, P, P, P, P, P, P, S, P]
     lib.dfs_block_score_pooled.argtypes = [sp, F, P, P, S, P]
+    lib.dfs_sparse_attn_lvsa_fwd.argtypes = [sp, P, P, P, P, P, I, F, ctypes.POINTER(_SelectParams), P, P, P]
     lib.dfs_sparse_attn_fwd.argtypes = [sp, P, P, P, P, P, I, F, P, P, P]
     lib.dfs_unperm.argtypes = [sp, P, P, P, P]
     lib.dfs_workspace_bytes.argtypes = [sp, I]
@@ -82,7 +83,7 @@ def _load():
     lib.dfs_version.argtypes = []
     for name in ("dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd",
                  "dfs_unperm", "dfs_get_error_flags", "dfs_version", "dfs_block_score_noalloc",
-                 "dfs_hilbert_perm_pooled", "dfs_block_score_pooled"):
+                 "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd"):
         getattr(lib, name).restype = I
     return lib
 
@@ -203,6 +204,14 @@ def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o
     _check("dfs_sparse_attn_fwd", LIB.dfs_sparse_attn_fwd(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
         _ptr(op), _ptr(lse), _stream(stream)))
+
+
+def dfs_sparse_attn_lvsa_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, params, op, lse=None,
+                             stream=None):
+    sh = shape.c()
+    _check("dfs_sparse_attn_lvsa_fwd", LIB.dfs_sparse_attn_lvsa_fwd(
+        ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
+        ctypes.byref(params), _ptr(op), _ptr(lse), _stream(stream)))
 
 
 def dfs_unperm(shape: Shape, perm, op, o, stream=None):

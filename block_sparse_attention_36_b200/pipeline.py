@@ -21,10 +21,15 @@ from . import dfsattn as lib
 class DfsLayer:
     def __init__(self, shape: lib.Shape, order="hilbert3d", mode="topk", k=0, cap=0, tau=0.0,
                  lvsa_T_per=8, lvsa_C=21, lvsa_step=0, kcap=None, scale=0.0, device="cuda",
-                 want_lse=False):
+                 want_lse=False, frame_exact=False):
         self.shape = shape
         self.order = order
         self.mode = mode
+        # LVSA only: drop the pairs of kept blocks whose key frame is outside
+        # A(t); frames must stay contiguous, so the order must be raster.
+        if frame_exact and (mode != "lvsa" or order != "raster"):
+            raise ValueError("frame_exact needs mode='lvsa' and order='raster'")
+        self.frame_exact = bool(frame_exact)
         self.params = lib.select_params(mode, k=k, cap=cap, tau=tau, lvsa_T_per=lvsa_T_per, lvsa_C=lvsa_C,
                                         lvsa_step=lvsa_step)
         s = shape
@@ -81,8 +86,12 @@ class DfsLayer:
         lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
 
     def attend(self, stream=None):
-        lib.dfs_sparse_attn_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt, self.kcap,
-                                self.scale, self.op, self.lse, stream)
+        if self.frame_exact:
+            lib.dfs_sparse_attn_lvsa_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt,
+                                         self.kcap, self.scale, self.params, self.op, self.lse, stream)
+        else:
+            lib.dfs_sparse_attn_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt, self.kcap,
+                                    self.scale, self.op, self.lse, stream)
         lib.dfs_unperm(self.shape, self.perm, self.op, self.out, stream)
 
     def permute_pooled(self, q, k, v, stream=None):

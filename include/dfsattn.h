@@ -212,6 +212,19 @@ int dfs_sparse_attn_fwd(const dfs_shape *shape, const void *qp, const void *kp, 
                         const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
                         void *op, float *lse, dfs_stream_t stream);
 
+/* dfs_sparse_attn_lvsa_fwd -- frame-exact LVSA attention (LVSA: Training-Free
+ * Sparse Attention for Long Video Diffusion, section 2).
+ *
+ * As dfs_sparse_attn_fwd over the kept blocks (normally the DFS_SEL_LVSA
+ * lists), and inside them every (query, key) pair whose key frame is not in
+ * the query frame's set A(t) (the rule of DFS_SEL_LVSA, from lvsa's T_per,
+ * C and step) is dropped, so each query attends exactly the frames of A(t).
+ * Requires raster order (curve order = raster) and H * W >= blk. A query row
+ * with no allowed key gets op = 0, lse = -inf.                             */
+int dfs_sparse_attn_lvsa_fwd(const dfs_shape *shape, const void *qp, const void *kp, const void *vp,
+                             const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
+                             const dfs_select_params *lvsa, void *op, float *lse, dfs_stream_t stream);
+
 /* dfs_unperm -- inverse reorder: o[b, perm[i], h, :] = op[b, h, i, :],
  * op bf16 [B, nh, N, D] (curve order) -> o bf16 [B, N, nh, D] (raster).   */
 int dfs_unperm(const dfs_shape *shape, const int32_t *perm, const void *op, void *o,

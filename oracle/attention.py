@@ -18,11 +18,13 @@ import math
 import numpy as np
 
 
-def block_sparse_attention(qp, kp, vp, kv_idx, kv_cnt, blk, scale=None, rows=None):
+def block_sparse_attention(qp, kp, vp, kv_idx, kv_cnt, blk, scale=None, rows=None, allowed=None):
     """O [B, nh, N, D] and lse [B, nh, N] over the kept blocks (curve order).
 
     ``rows`` optionally restricts the work to a list of (b, h, I) query
-    blocks; the other outputs are left as NaN.
+    blocks; the other outputs are left as NaN. ``allowed(q_pos, k_pos)``
+    optionally drops (query, key) pairs inside the kept blocks: it maps
+    arrays of query and key positions to a boolean matrix.
     """
     q = np.asarray(qp, dtype=np.float64)
     k = np.asarray(kp, dtype=np.float64)
@@ -45,6 +47,8 @@ def block_sparse_attention(qp, kp, vp, kv_idx, kv_cnt, blk, scale=None, rows=Non
             continue
         ks = np.concatenate(keys)
         s = (q[b, h, q_lo:q_hi] @ k[b, h, ks].T) * scale
+        if allowed is not None:
+            s = np.where(allowed(np.arange(q_lo, q_hi), ks), s, -np.inf)
         m = s.max(axis=1, keepdims=True)
         e = np.exp(s - m)
         z = e.sum(axis=1, keepdims=True)

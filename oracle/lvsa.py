@@ -18,7 +18,10 @@ Readings:
     P = H * W tokens;
   * key block J is kept for query block I when some frame touched by J lies
     in the union of A(t) over the frames t touched by I. Attention is then
-    exact for this block mask.
+    exact for this block mask;
+  * frame-exact attention additionally drops, inside the kept blocks, every
+    (query, key) pair whose key frame is not in A(query frame), so the
+    attended set is exactly A(t) (frame_allowed).
 """
 from __future__ import annotations
 
@@ -69,4 +72,12 @@ def block_mask(T, P, blk, T_per, C, s):
             allowed |= A[t]
         for J in range(nb):
             m[I, J] = any(f in allowed for f in block_frames(J, blk, N, P))
+    return m
+
+
+def frame_allowed(T, T_per, C, s):
+    """Boolean [T, T]: query frame t may attend key frame f iff f in A(t)."""
+    m = np.zeros((T, T), dtype=bool)
+    for t in range(T):
+        m[t, frame_set(T, t, T_per, C, s)] = True
     return m

@@ -194,6 +194,7 @@ class Workload:
     lvsa_step: int = 0
     n_steps: int = 0
     refresh: int = 0
+    frame_exact: bool = False   # LVSA: mask pairs outside A(t) inside kept blocks
 
     @property
     def N(self):
@@ -223,6 +224,8 @@ WORKLOADS = {
                                 n_steps=50, refresh=5),
     "lvsa_long_video": Workload("lvsa_long_video", 1, 12, 128, 63, 30, 52, 128, 32, "raster", "lvsa",
                                 lvsa_T_per=8, lvsa_C=21, lvsa_step=0),
+    "lvsa_long_video_exact": Workload("lvsa_long_video_exact", 1, 12, 128, 63, 30, 52, 128, 32, "raster", "lvsa",
+                                      lvsa_T_per=8, lvsa_C=21, lvsa_step=0, frame_exact=True),
     "wan_1p3b_global": Workload("wan_1p3b_global", 1, 12, 128, 21, 30, 52, 128, 32, "hilbert3d", "global",
                                 keep_num=15),
     "hunyuan_layer": Workload("hunyuan_layer", 1, 24, 128, 33, 45, 80, 128, 32, "hilbert3d", "threshold",

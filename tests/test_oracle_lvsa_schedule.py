@@ -88,3 +88,24 @@ def test_schedule_closed_form():
     for s in range(1, 50):
         if ks[s] != ks[s - 1]:
             assert schedule.is_refresh(s)
+
+
+def test_frame_exact_attention_toy():
+    # token-level brute force on a 5-frame toy (P = 6, blk 4): frame-exact
+    # attention equals dense attention restricted to A(t) frame by frame
+    from oracle import attention, selection
+    T, P, blk, T_per, C, s = 5, 6, 4, 3, 3, 1
+    N = T * P
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.standard_normal((1, 1, N, 4)) for _ in range(3))
+    m = lvsa.block_mask(T, P, blk, T_per, C, s)
+    idx, cnt = selection.mask_to_lists(m[None, None])
+    fa = lvsa.frame_allowed(T, T_per, C, s)
+    allowed = lambda qs, ks: fa[np.asarray(qs)[:, None] // P, np.asarray(ks)[None, :] // P]
+    got, _ = attention.block_sparse_attention(q, k, v, idx, cnt, blk, 0.5, allowed=allowed)
+    for n in range(N):
+        keys = [j for j in range(N) if fa[n // P, j // P]]
+        lg = np.array([0.5 * float(q[0, 0, n] @ k[0, 0, j]) for j in keys])
+        e = np.exp(lg - lg.max())
+        ref = (e[:, None] * v[0, 0, keys]).sum(0) / e.sum()
+        assert np.abs(got[0, 0, n] - ref).max() < 1e-12
