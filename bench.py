@@ -37,14 +37,14 @@ if ROOT not in sys.path:
 
 METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
 # fused gather + pooling (1 launch), score, select, attention, scatter; LVSA: 3 gathers, select, attention, scatter
-KERNELS_PER_STEP = {"topk": 5, "threshold": 5, "global": 5, "lvsa": 6}
+KERNELS_PER_STEP = {"topk": 5, "threshold": 5, "global": 5, "lvsa": 6, "radial": 6}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per attention launch from one ncu capture
 # (profiles/attn_fwd_<workload>.md), valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
-ATTN_TRAFFIC = {"wan_1p3b_layer": (297_903_360 + 82_006_784, "008d78ef19061aff")}
-ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh")
+ATTN_TRAFFIC = {"wan_1p3b_layer": (297_875_968 + 84_863_488, "fe92b8f843351e08")}
+ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh")
 
 
 def attn_sources_hash():
@@ -75,7 +75,9 @@ def load_peaks():
 def workload_config(wl, k, cap):
     sel = {"topk": f"top-k {k}/{wl.nb}", "threshold": f"threshold tau={wl.tau} cap {cap}/{wl.nb}",
            "global": f"global top {k} of {wl.nb}x{wl.nb} pairs per head",
-           "lvsa": f"LVSA T_per={wl.lvsa_T_per} C={wl.lvsa_C} step {wl.lvsa_step}"}[wl.mode]
+           "lvsa": f"LVSA T_per={wl.lvsa_T_per} C={wl.lvsa_C} step {wl.lvsa_step}"
+                   + (" frame-exact" if wl.frame_exact else ""),
+           "radial": f"log-radial w0={wl.radial_w0} lambda={wl.radial_lambda}"}[wl.mode]
     return (f"{wl.name}: B={wl.B} nh={wl.nh} D={wl.D} grid {wl.T}x{wl.H}x{wl.W} (N={wl.N}) "
             f"{wl.order} order, blk {wl.blk}, sb {wl.sb}, {sel}")
 
@@ -192,6 +194,9 @@ def make_layer(bsa, wl):
     elif wl.mode == "global":
         k = wl.pair_count(wl.keep_num)
         layer = bsa.DfsLayer(s, order=wl.order, mode="global", k=k, kcap=s.nb)
+    elif wl.mode == "radial":
+        layer = bsa.DfsLayer(s, order=wl.order, mode="radial", radial_w0=wl.radial_w0,
+                             radial_lambda=wl.radial_lambda)
     else:
         layer = bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
                              lvsa_step=wl.lvsa_step, frame_exact=wl.frame_exact)
@@ -242,8 +247,7 @@ def run_ours(args):
             continue
         layer.prepare(q, k, v)
         ev_attn[i][0].record(stream)
-        dfsattn.dfs_sparse_attn_fwd(layer.shape, layer.qp, layer.kp, layer.vp, layer.kv_idx, layer.kv_cnt,
-                                    layer.kcap, layer.scale, layer.op, None)
+        layer.attention()
         ev_attn[i][1].record(stream)
         dfsattn.dfs_unperm(layer.shape, layer.perm, layer.op, layer.out)
     stop.record(stream)
@@ -255,8 +259,7 @@ def run_ours(args):
         # attention-kernel time from eager launches (events cannot sit inside the graph replay)
         for i in range(args.steps):
             ev_attn[i][0].record(stream)
-            dfsattn.dfs_sparse_attn_fwd(layer.shape, layer.qp, layer.kp, layer.vp, layer.kv_idx, layer.kv_cnt,
-                                        layer.kcap, layer.scale, layer.op, None)
+            layer.attention()
             ev_attn[i][1].record(stream)
         torch.cuda.synchronize()
         del graph
@@ -413,7 +416,7 @@ def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, steps=1):
     budget; the time per query block is scaled to the whole layer.
     Returns the oracle's whole-step throughput in the same unit."""
     import torch
-    from oracle import attention, hilbert, lvsa, scoring, selection
+    from oracle import attention, hilbert, lvsa, radial, scoring, selection
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     t0 = time.perf_counter()
     perm, _ = hilbert.make_perm(wl.order, wl.T, wl.H, wl.W)
@@ -430,6 +433,10 @@ def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, steps=1):
         qp, kp, vp = (qkv[n][0, permt, h, :].double().numpy()[None, None] for n in ("q", "k", "v"))
         if wl.mode == "lvsa":
             m = lvsa.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step) if h == 0 else m
+            idx, cnt = selection.mask_to_lists(m[None, None])
+        elif wl.mode == "radial":
+            m = radial.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.radial_w0,
+                                  radial.w_far_of(wl.radial_lambda, wl.radial_w0)) if h == 0 else m
             idx, cnt = selection.mask_to_lists(m[None, None])
         else:
             sc = scoring.block_scores(qp, kp, wl.blk, wl.sb)

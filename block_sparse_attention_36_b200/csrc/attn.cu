@@ -169,7 +169,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const bool ok = (j < cnt) && J >= 0 && J < nb;
         bad |= (j < cnt) && !ok;
         const unsigned m = __ballot_sync(0xffffffffu, ok);
-        if (ok) dst[base + __popc(m & ((1u << lane) - 1u))] = J;
+        if (ok) {
+          const int pos = base + __popc(m & ((1u << lane) - 1u));
+          dst[pos] = J;
+          if (FRAME) {
+            // first frame of the key block and the columns that lie in it
+            const int k0 = J * BLK;
+            const int f0 = k0 / fm.P;
+            const int cb = min(BLK, (f0 + 1) * fm.P - k0);
+            dst[2 * max_list + pos] = (f0 << 8) | cb;
+          }
+        }
         base += __popc(m);
       }
     }
@@ -177,7 +187,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0) bars->n_kv[x] = base;
   }
   if (warp == 1) tmem_alloc(&bars->tmem_base, C::kTmemCols);
-  uint32_t* ftab = reinterpret_cast<uint32_t*>(lists + 2 * max_list);
+  // FRAME only: per list entry (first key frame << 8 | columns in it), then the frame bit sets
+  const int32_t* kmeta = lists + 2 * max_list;
+  uint32_t* ftab = reinterpret_cast<uint32_t*>(lists + 4 * max_list);
   const int qf_lo = FRAME ? (I0 * BLK) / fm.P : 0;
   if (FRAME && warp >= 4) {
     const int words = frame_words(fm.T);
@@ -341,9 +353,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (FRAME) {
         // Keys of this block lie in frames f0 (columns < cb) and f0 + 1;
         // drop the frame(s) outside A(query frame).
-        const int k0 = list[j] * BLK;
-        const int f0 = k0 / fm.P;
-        const int cb = min(BLK, (f0 + 1) * fm.P - k0);
+        const int mt = kmeta[x * max_list + j];
+        const int f0 = mt >> 8, cb = mt & 255;
         const bool a0 = (frow[f0 >> 5] >> (f0 & 31)) & 1u;
         const bool a1 = cb >= BLK || (f0 + 1 < fm.T && ((frow[(f0 + 1) >> 5] >> ((f0 + 1) & 31)) & 1u));
         if (!a0 || !a1) {
@@ -514,7 +525,7 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
     return DFS_ERR_CUDA;
   const int max_list = min(kcap, d.nb);
   size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + 2 * (size_t)max_list * sizeof(int32_t);
-  if (FRAME) smem += (size_t)kFrameRows * frame_words(fm.T) * sizeof(uint32_t);
+  if (FRAME) smem += 2 * (size_t)max_list * sizeof(int32_t) + (size_t)kFrameRows * frame_words(fm.T) * sizeof(uint32_t);
   if (smem > 232448) return DFS_ERR_UNSUPPORTED;
   // Tensor memory per SM is 512 columns: a 512-column CTA must be alone on
   // its SM and a 256-column CTA may share it with one other, so shared

@@ -213,6 +213,62 @@ select_lvsa_kernel(int rows, int nb, long long N, int blk, int P, int T, int T_p
   }
 }
 
+// Log-radial static mask (DynamicRad, methodology, components 1 and 2):
+// query token q may attend key token k iff 2 |s_q - s_k| < omega(d), with
+// d the frame distance, s the spatial index in the frame and
+// omega(d) = max(w0 >> bitlength(d), w_far). Key block J is kept for query
+// block I iff some pair qualifies. Each block splits into per-frame
+// segments of spatial indices; two segments have a qualifying pair iff the
+// gap between their index intervals is small enough, so a block pair costs
+// (segments of I) x (segments of J) tests (2 x 2 when H*W >= blk).
+__device__ __forceinline__ bool radial_segments_meet(int t, int a0, int a1, int f, int b0, int b1, int w0,
+                                                     int w_far) {
+  const unsigned d = (unsigned)(t > f ? t - f : f - t);
+  const int band = 32 - __clz((int)d);
+  const int om = max(band >= 31 ? 0 : (w0 >> band), w_far);
+  const int gap = max(0, max(b0 - a1, a0 - b1));
+  return 2LL * gap < (long long)om;
+}
+
+__global__ void __launch_bounds__(256)
+select_radial_kernel(int rows, int nb, long long N, int blk, int P, int w0, int w_far,
+                     int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, int kcap) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int I = (int)(row % nb);
+  const long long q_lo = (long long)I * blk, q_hi = min(q_lo + blk, N) - 1;
+  const int qf0 = (int)(q_lo / P), qf1 = (int)(q_hi / P);
+  int32_t* out = kv_idx + row * (long long)kcap;
+  const unsigned lt = (1u << lane) - 1u;
+  int base = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int J = j0 + lane;
+    bool take = false;
+    if (J < nb) {
+      const long long k_lo = (long long)J * blk, k_hi = min(k_lo + blk, N) - 1;
+      const int kf0 = (int)(k_lo / P), kf1 = (int)(k_hi / P);
+      for (int t = qf0; t <= qf1 && !take; ++t) {
+        const long long tb = (long long)t * P;
+        const int a0 = (int)(max(q_lo, tb) - tb), a1 = (int)(min(q_hi, tb + P - 1) - tb);
+        for (int f = kf0; f <= kf1 && !take; ++f) {
+          const long long fb = (long long)f * P;
+          const int b0 = (int)(max(k_lo, fb) - fb), b1 = (int)(min(k_hi, fb + P - 1) - fb);
+          take = radial_segments_meet(t, a0, a1, f, b0, b1, w0, w_far);
+        }
+      }
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = base + __popc(tb & lt);
+    if (take && pos < kcap) out[pos] = J;
+    base += __popc(tb);
+  }
+  if (lane == 0) {
+    if (base > kcap) atomicOr(&g_select_flags, (uint32_t)DFS_FLAG_KCAP_OVERFLOW);
+    kv_cnt[row] = min(base, kcap);
+  }
+}
+
 // Global selection (VMoBA, abstract, modification 2): per head (one CTA),
 // the K best (query block, key block) pairs of all nb x nb, equal scores to
 // the lower flat index I * nb + J; rows list their kept J ascending.
@@ -324,6 +380,16 @@ extern "C" int dfs_select_mask(const dfs_shape* shape, const float* scores, cons
     select_lvsa_kernel<<<grid, 256, 0, cs>>>((int)rows, d.nb, d.N, d.blk, (int)P, d.T, prm->lvsa_T_per,
                                              prm->lvsa_C, prm->lvsa_step % prm->lvsa_T_per, kv_idx,
                                              kv_cnt, kcap);
+    return dfs::launch_status();
+  }
+  if (prm->mode == DFS_SEL_RADIAL) {
+    const long long P = (long long)d.H * d.W;
+    const double lam = (double)prm->radial_lambda;
+    if (prm->radial_w0 < 0 || !(lam >= 0.0) || lam > 1e9) return DFS_ERR_INVALID_ARG;
+    const double wf = floor(lam * (double)prm->radial_w0);
+    const int w_far = wf >= 2147483647.0 ? 2147483647 : (int)wf;
+    select_radial_kernel<<<grid, 256, 0, cs>>>((int)rows, d.nb, d.N, d.blk, (int)P, prm->radial_w0, w_far,
+                                               kv_idx, kv_cnt, kcap);
     return dfs::launch_status();
   }
   if (!scores) return DFS_ERR_INVALID_ARG;

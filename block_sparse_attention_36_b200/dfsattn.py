@@ -30,6 +30,7 @@ DFS_SEL_TOPK = 0
 DFS_SEL_THRESHOLD = 1
 DFS_SEL_LVSA = 2
 DFS_SEL_GLOBAL = 3
+DFS_SEL_RADIAL = 4
 DFS_WS_BLOCK_SCORE = 0
 
 DFS_FLAG_WAIT_TIMEOUT = 1
@@ -40,7 +41,8 @@ DFS_ORDER_TILE2D = 2
 DFS_ORDER_TILE3D = 3
 ORDERS = {"raster": DFS_ORDER_RASTER, "hilbert3d": DFS_ORDER_HILBERT3D, "tile2d": DFS_ORDER_TILE2D,
           "tile3d": DFS_ORDER_TILE3D}
-MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA, "global": DFS_SEL_GLOBAL}
+MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA, "global": DFS_SEL_GLOBAL,
+         "radial": DFS_SEL_RADIAL}
 
 # C entry points declared in include/dfsattn.h.
 EXPORTS = (
@@ -56,7 +58,8 @@ class _Shape(ctypes.Structure):
 
 class _SelectParams(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("k", ctypes.c_int), ("cap", ctypes.c_int), ("tau", ctypes.c_float),
-                ("lvsa_T_per", ctypes.c_int), ("lvsa_C", ctypes.c_int), ("lvsa_step", ctypes.c_int)]
+                ("lvsa_T_per", ctypes.c_int), ("lvsa_C", ctypes.c_int), ("lvsa_step", ctypes.c_int),
+                ("radial_w0", ctypes.c_int), ("radial_lambda", ctypes.c_float)]
 
 
 def _load():
@@ -187,9 +190,10 @@ def dfs_block_score_noalloc(shape: Shape, qp, kp, scale, scores, stream=None):
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
-def select_params(mode, k=0, cap=0, tau=0.0, lvsa_T_per=8, lvsa_C=21, lvsa_step=0):
+def select_params(mode, k=0, cap=0, tau=0.0, lvsa_T_per=8, lvsa_C=21, lvsa_step=0, radial_w0=0,
+                  radial_lambda=0.0):
     return _SelectParams(MODES.get(mode, mode), int(k), int(cap), float(tau), int(lvsa_T_per), int(lvsa_C),
-                         int(lvsa_step))
+                         int(lvsa_step), int(radial_w0), float(radial_lambda))
 
 
 def dfs_select_mask(shape: Shape, scores, params, kv_idx, kv_cnt, kcap, stream=None):

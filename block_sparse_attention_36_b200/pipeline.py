@@ -18,10 +18,14 @@ import torch
 from . import dfsattn as lib
 
 
+# selection modes whose mask needs no block scores
+STATIC_MODES = ("lvsa", "radial")
+
+
 class DfsLayer:
     def __init__(self, shape: lib.Shape, order="hilbert3d", mode="topk", k=0, cap=0, tau=0.0,
                  lvsa_T_per=8, lvsa_C=21, lvsa_step=0, kcap=None, scale=0.0, device="cuda",
-                 want_lse=False, frame_exact=False):
+                 want_lse=False, frame_exact=False, radial_w0=0, radial_lambda=0.0):
         self.shape = shape
         self.order = order
         self.mode = mode
@@ -31,7 +35,7 @@ class DfsLayer:
             raise ValueError("frame_exact needs mode='lvsa' and order='raster'")
         self.frame_exact = bool(frame_exact)
         self.params = lib.select_params(mode, k=k, cap=cap, tau=tau, lvsa_T_per=lvsa_T_per, lvsa_C=lvsa_C,
-                                        lvsa_step=lvsa_step)
+                                        lvsa_step=lvsa_step, radial_w0=radial_w0, radial_lambda=radial_lambda)
         s = shape
         if kcap is None:
             kcap = {"topk": max(1, min(k, s.nb)), "threshold": max(1, min(cap, s.nb)),
@@ -50,7 +54,7 @@ class DfsLayer:
         self.lse = torch.empty((s.B, s.nh, s.N), dtype=torch.float32, device=dev) if want_lse else None
         self.kv_idx = torch.full((s.B, s.nh, s.nb, self.kcap), -1, dtype=torch.int32, device=dev)
         self.kv_cnt = torch.zeros((s.B, s.nh, s.nb), dtype=torch.int32, device=dev)
-        if mode != "lvsa":
+        if mode not in STATIC_MODES:
             self.scores = torch.empty((s.B, s.nh, s.nb, s.nb), dtype=torch.float32, device=dev)
             nbytes = lib.dfs_workspace_bytes(s, lib.DFS_WS_BLOCK_SCORE)
             self.ws = torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev)
@@ -81,18 +85,22 @@ class DfsLayer:
         self._index_built = True
 
     def build_mask(self, stream=None):
-        if self.mode != "lvsa":
+        if self.mode not in STATIC_MODES:
             lib.dfs_block_score(self.shape, self.qp, self.kp, self.scale, self.scores, self.ws, stream)
         lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
 
     def attend(self, stream=None):
+        self.attention(stream)
+        lib.dfs_unperm(self.shape, self.perm, self.op, self.out, stream)
+
+    def attention(self, stream=None):
+        """The attention kernel alone (curve order, into ``op``)."""
         if self.frame_exact:
             lib.dfs_sparse_attn_lvsa_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt,
                                          self.kcap, self.scale, self.params, self.op, self.lse, stream)
         else:
             lib.dfs_sparse_attn_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt, self.kcap,
                                     self.scale, self.op, self.lse, stream)
-        lib.dfs_unperm(self.shape, self.perm, self.op, self.out, stream)
 
     def permute_pooled(self, q, k, v, stream=None):
         """Reorder Q, K, V and pool Q, K into the score workspace in one pass."""
@@ -104,7 +112,7 @@ class DfsLayer:
         """Reorder Q, K, V and, if asked, rebuild the mask. When the mask is
         rebuilt from scores, the reorder also pools Q and K (one pass over the
         data) and scoring starts from those means."""
-        if refresh_mask and self.mode != "lvsa" and self.fused_pool:
+        if refresh_mask and self.mode not in STATIC_MODES and self.fused_pool:
             self.permute_pooled(q, k, v, stream)
             lib.dfs_block_score_pooled(self.shape, self.scale, self.scores, self.ws, stream)
             lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)

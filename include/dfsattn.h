@@ -63,7 +63,7 @@ typedef struct {
 } dfs_shape;
 
 enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1, DFS_ORDER_TILE2D = 2, DFS_ORDER_TILE3D = 3 };
-enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2, DFS_SEL_GLOBAL = 3 };
+enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2, DFS_SEL_GLOBAL = 3, DFS_SEL_RADIAL = 4 };
 enum { DFS_WS_BLOCK_SCORE = 0 };
 
 /* Device error word bits (dfs_get_error_flags). */
@@ -94,13 +94,26 @@ enum {
  *                              scores: lower flat index I * nb + J first);
  *                              each query block lists its kept key blocks
  *                              ascending and may keep none. k counts pairs
- *                              per head here.                                  */
+ *                              per head here.
+ *   mode = DFS_SEL_RADIAL    : scores ignored (may be NULL). Log-radial
+ *                              static mask of DynamicRad (methodology,
+ *                              components 1 and 2; static-ratio mode), raster
+ *                              order, frames of P = H*W tokens: query token q
+ *                              may attend key token k iff
+ *                              2 |s_q - s_k| < max(w0 >> bitlen(d), w_far),
+ *                              d = |frame(q) - frame(k)|, s = index inside
+ *                              the frame, w0 = radial_w0 (>= 0) and
+ *                              w_far = floor((double)radial_lambda * w0)
+ *                              (radial_lambda >= 0). Key block J is kept
+ *                              for query block I when some pair qualifies. */
 typedef struct {
   int mode;
   int k;
   int cap;
   float tau;
   int lvsa_T_per, lvsa_C, lvsa_step;
+  int radial_w0;
+  float radial_lambda;
 } dfs_select_params;
 
 /* dfs_hilbert_perm -- token reorder (DFSAttn, Methodology item 1).
@@ -184,7 +197,8 @@ int dfs_block_score_noalloc(const dfs_shape *shape, const void *qp, const void *
 /* dfs_select_mask -- key-block selection (DFSAttn, Methodology item 3;
  * VMoBA abstract, modification 3; LVSA section 2).
  *
- * scores: fp32 [B, nh, nb, nb] (NULL allowed for DFS_SEL_LVSA).
+ * scores: fp32 [B, nh, nb, nb] (NULL allowed for DFS_SEL_LVSA and
+ * DFS_SEL_RADIAL).
  * Writes, per row (b, h, I), the kept key-block indices in ascending order
  * to kv_idx[((b*nh + h)*nb + I)*kcap + 0 .. cnt-1] (int32) and cnt to
  * kv_cnt[(b*nh + h)*nb + I]. Slots past cnt are not written. kcap >= 1; for

@@ -185,7 +185,7 @@ class Workload:
     blk: int
     sb: int
     order: str            # "hilbert3d" or "raster"
-    mode: str             # "topk", "threshold", "lvsa", "schedule", "global"
+    mode: str             # "topk", "threshold", "lvsa", "schedule", "global", "radial"
     keep_num: int = 0     # keep ratio numerator / 100 (top-k)
     tau: float = 0.0
     cap_num: int = 0      # cap ratio numerator / 100 (threshold)
@@ -195,6 +195,8 @@ class Workload:
     n_steps: int = 0
     refresh: int = 0
     frame_exact: bool = False   # LVSA: mask pairs outside A(t) inside kept blocks
+    radial_w0: int = 0          # log-radial mask: window at frame distance 0 (tokens)
+    radial_lambda: float = 0.0  # log-radial mask: long-range floor, as a fraction of w0
 
     @property
     def N(self):
@@ -226,6 +228,8 @@ WORKLOADS = {
                                 lvsa_T_per=8, lvsa_C=21, lvsa_step=0),
     "lvsa_long_video_exact": Workload("lvsa_long_video_exact", 1, 12, 128, 63, 30, 52, 128, 32, "raster", "lvsa",
                                       lvsa_T_per=8, lvsa_C=21, lvsa_step=0, frame_exact=True),
+    "wan_1p3b_radial": Workload("wan_1p3b_radial", 1, 12, 128, 21, 30, 52, 128, 32, "raster", "radial",
+                                radial_w0=1560, radial_lambda=0.125),
     "wan_1p3b_global": Workload("wan_1p3b_global", 1, 12, 128, 21, 30, 52, 128, 32, "hilbert3d", "global",
                                 keep_num=15),
     "hunyuan_layer": Workload("hunyuan_layer", 1, 24, 128, 33, 45, 80, 128, 32, "hilbert3d", "threshold",

@@ -2,15 +2,16 @@
 
 Pages: DFSAttn, Methodology item 3 (top-k budget); VMoBA abstract,
 modifications (2) (global selection) and (3) (cumulative-mass threshold);
-LVSA section 2 (frame mask). Given the same fp32 scores, top-k and global
-lists are bit-exact (ties included); a threshold row may differ only where
-the oracle's cumulative mass at the cut lies within 1e-5 of tau (counted);
-LVSA lists are bit-exact."""
+LVSA section 2 (frame mask); DynamicRad methodology (log-radial static
+mask). Given the same fp32 scores, top-k and global lists are bit-exact
+(ties included); a threshold row may differ only where the oracle's
+cumulative mass at the cut lies within 1e-5 of tau (counted); LVSA and
+log-radial lists are bit-exact."""
 import numpy as np
 import pytest
 import torch
 
-from oracle import lvsa, selection
+from oracle import lvsa, radial, selection
 from tests.parity import compare_masks
 
 pytestmark = pytest.mark.gpu
@@ -93,6 +94,35 @@ def test_lvsa_bit_exact(lib, T, H, W, blk, T_per, C):
         m = lvsa.block_mask(T, H * W, blk, T_per, C, s)
         oi, oc = selection.mask_to_lists(np.broadcast_to(m, (1, nh) + m.shape), kcap)
         _lists_equal(gi, gc, oi, oc)
+
+
+@pytest.mark.parametrize("T,H,W,blk,w0,lam", [
+    (6, 4, 5, 64, 12, 0.2),        # frames smaller than a block (P = 20 < 64)
+    (9, 7, 1, 64, 20, 0.0),        # P = 7, many frames per block
+    (5, 8, 9, 64, 144, 0.0625),    # P = 72, window of a whole frame at d = 0
+    (8, 5, 8, 64, 40, 0.15),       # P = 40 < blk = 64
+    (11, 16, 12, 128, 192, 0.125), # P = 1.5 blk
+    (7, 10, 13, 128, 1, 0.0),      # w0 = 1: only equal positions in the same frame
+    (5, 12, 12, 64, 288, 1.0),     # window 2P everywhere: dense
+])
+def test_radial_bit_exact(lib, T, H, W, blk, w0, lam):
+    nh = 2
+    shape = lib.Shape(1, nh, 128, T, H, W, blk, 32)
+    kcap = shape.nb
+    gi, gc = _select(lib, None, shape, lib.select_params("radial", radial_w0=w0, radial_lambda=lam), kcap)
+    m = radial.block_mask(T, H * W, blk, w0, radial.w_far_of(lam, w0))
+    oi, oc = selection.mask_to_lists(np.broadcast_to(m, (1, nh) + m.shape), kcap)
+    _lists_equal(gi, gc, oi, oc)
+
+
+def test_radial_wan_grid_sampled_rows(lib):
+    T, H, W, blk, w0, lam = 21, 30, 52, 128, 1560, 0.125
+    shape = lib.Shape(1, 1, 128, T, H, W, blk, 32)
+    gi, gc = _select(lib, None, shape, lib.select_params("radial", radial_w0=w0, radial_lambda=lam), shape.nb)
+    rows = [0, 1, 12, 13, 100, 127, 128, 200, 254, 255]
+    m = radial.block_mask(T, H * W, blk, w0, radial.w_far_of(lam, w0), rows=rows)
+    for r, I in enumerate(rows):
+        assert np.array_equal(gi[0, 0, I, :gc[0, 0, I]], np.flatnonzero(m[r])), I
 
 
 def test_kcap_overflow_is_flagged(lib):

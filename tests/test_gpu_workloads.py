@@ -1,4 +1,4 @@
-"""The whole path on the five synthetic workloads against the oracle.
+"""The whole path on the synthetic workloads against the oracle.
 
 * permutation: bit-exact;
 * block scores: fp32 against fp64 within the rounding bound;
@@ -18,7 +18,7 @@ import pytest
 import torch
 
 import synth
-from oracle import attention, hilbert, lvsa, pipeline, schedule, scoring, selection
+from oracle import attention, hilbert, lvsa, pipeline, radial, schedule, scoring, selection
 from tests.parity import assert_attn_close, compare_global_masks, compare_masks
 
 pytestmark = pytest.mark.gpu
@@ -40,6 +40,9 @@ def _layer(bsa, wl, **kw):
     if wl.mode == "lvsa":
         return bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
                             lvsa_step=wl.lvsa_step, want_lse=True, **kw)
+    if wl.mode == "radial":
+        return bsa.DfsLayer(s, order=wl.order, mode="radial", radial_w0=wl.radial_w0,
+                            radial_lambda=wl.radial_lambda, want_lse=True, **kw)
     if wl.mode == "global":
         return bsa.DfsLayer(s, order=wl.order, mode="global", k=wl.pair_count(wl.keep_num), kcap=s.nb,
                             want_lse=True, **kw)
@@ -108,7 +111,8 @@ def test_tiny_workload_end_to_end(bsa):
     assert_attn_close(out, hilbert.unpermute_tokens(full, res["perm"]), "tiny output, GPU lists")
 
 
-@pytest.mark.parametrize("name", ["wan_1p3b_layer", "hunyuan_layer", "lvsa_long_video", "wan_1p3b_global"])
+@pytest.mark.parametrize("name", ["wan_1p3b_layer", "hunyuan_layer", "lvsa_long_video", "wan_1p3b_global",
+                                  "wan_1p3b_radial"])
 def test_full_size_workload(bsa, name):
     wl = synth.WORKLOADS[name]
     qkv = synth.workload_inputs(wl)
@@ -125,6 +129,15 @@ def test_full_size_workload(bsa, name):
         gi = layer.kv_idx.cpu().numpy()
         for idx in np.ndindex(oc.shape):
             assert np.array_equal(gi[idx][:oc[idx]], oi[idx][:oc[idx]])
+    elif wl.mode == "radial":
+        rows = [0, 5, 77, 128, 191, wl.nb - 1]
+        m = radial.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.radial_w0, radial.w_far_of(wl.radial_lambda, wl.radial_w0),
+                              rows=rows)
+        gi, gc = layer.kv_idx.cpu().numpy(), layer.kv_cnt.cpu().numpy()
+        for b in range(wl.B):
+            for h in range(wl.nh):
+                for r, I in enumerate(rows):
+                    assert np.array_equal(gi[b, h, I, :gc[b, h, I]], np.flatnonzero(m[r]))
     else:
         ref_scores = _oracle_scores(qkv["q"], qkv["k"], operm, wl)
         got_scores = layer.scores.cpu().numpy()
