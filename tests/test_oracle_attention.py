@@ -124,3 +124,54 @@ def test_recall_closed_forms():
     e = np.exp(np.array(s) - max(s))
     ref = e[perm[:blk]].sum() / e.sum()
     assert abs(recall.recall(q, k, perm, one, ones, blk, [(0, 0, n)]) - ref) < 1e-12
+
+
+def _loss(q, k, v, do, idx, cnt, blk, scale):
+    o, _ = attention.block_sparse_attention(q, k, v, idx, cnt, blk, scale)
+    return float((o * do).sum())
+
+
+def test_backward_matches_finite_differences():
+    # L = sum(dO * O); central differences of the forward oracle, element by element
+    B, nh, N, D, blk, scale = 1, 1, 19, 3, 8, 0.7
+    rng = np.random.default_rng(11)
+    q, k, v, do = (rng.standard_normal((B, nh, N, D)) for _ in range(4))
+    idx = np.array([[[[0, 2], [1, -1], [0, 1]]]], dtype=np.int32)   # block 2 is ragged (3 keys)
+    cnt = np.array([[[2, 1, 2]]], dtype=np.int32)
+    dq, dk, dv = attention.block_sparse_attention_bwd(q, k, v, do, idx, cnt, blk, scale)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for pos in np.ndindex(x.shape):
+            old = x[pos]
+            x[pos] = old + h
+            lp = _loss(q, k, v, do, idx, cnt, blk, scale)
+            x[pos] = old - h
+            lm = _loss(q, k, v, do, idx, cnt, blk, scale)
+            x[pos] = old
+            assert abs((lp - lm) / (2 * h) - g[pos]) < 1e-7, (name, pos)
+
+
+def test_backward_full_mask_matches_autograd():
+    import torch
+    B, nh, N, D, blk = 1, 2, 21, 4, 8
+    q, k, v, do = _qkv(B, nh, N, D, 12) + [np.random.default_rng(13).standard_normal((B, nh, N, D))]
+    nb = -(-N // blk)
+    idx, cnt = _full_lists(B, nh, nb)
+    dq, dk, dv = attention.block_sparse_attention_bwd(q, k, v, do, idx, cnt, blk)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    o = torch.softmax(tq @ tk.transpose(-1, -2) / math.sqrt(D), dim=-1) @ tv
+    o.backward(torch.tensor(do))
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(mine - ref.numpy()).max() < 1e-12
+
+
+def test_backward_empty_row_contributes_nothing():
+    q, k, v, do = _qkv(1, 1, 16, 4, 14) + [np.ones((1, 1, 16, 4))]
+    idx = np.array([[[[0], [0]]]], dtype=np.int32)
+    cnt = np.array([[[0, 1]]], dtype=np.int32)
+    dq, dk, dv = attention.block_sparse_attention_bwd(q, k, v, do, idx, cnt, 8)
+    assert (dq[0, 0, :8] == 0).all()
+    # only query block 1 reaches key block 0; key block 1 is never kept
+    assert (dk[0, 0, 8:] == 0).all() and (dv[0, 0, 8:] == 0).all()
+    ref_q, ref_k, ref_v = attention.block_sparse_attention_bwd(q, k, v, do, idx, cnt, 8, rows=[(0, 0, 1)])
+    assert np.array_equal(dk, ref_k) and np.array_equal(dv, ref_v)
