@@ -16,6 +16,11 @@ is the maximum over ranks.
 
 --impl reference times the fp64 CPU oracle (the only reference this
 method has) on the host cores over a bounded sample of the same workload.
+
+--backward times the gradient pass instead: after one forward, each step is
+DfsLayer.backward (reorder dO, the block-sparse attention backward, scatter
+dQ, dK, dV back); metric: kept-block TFLOP/s at 10 * D FLOPs per kept pair
+(the five products of the backward; the implementation executes seven).
 """
 from __future__ import annotations
 
@@ -182,24 +187,24 @@ def sum_over_ranks(x, world):
     return float(t.item())
 
 
-def make_layer(bsa, wl):
+def make_layer(bsa, wl, want_lse=False):
     s = bsa.Shape(wl.B, wl.nh, wl.D, wl.T, wl.H, wl.W, wl.blk, wl.sb)
     k = cap = 0
+    kw = {"order": wl.order, "want_lse": want_lse}
     if wl.mode == "topk":
         k = wl.ratio_count(wl.keep_num)
-        layer = bsa.DfsLayer(s, order=wl.order, mode="topk", k=k)
+        layer = bsa.DfsLayer(s, mode="topk", k=k, **kw)
     elif wl.mode == "threshold":
         cap = wl.ratio_count(wl.cap_num)
-        layer = bsa.DfsLayer(s, order=wl.order, mode="threshold", cap=cap, tau=wl.tau)
+        layer = bsa.DfsLayer(s, mode="threshold", cap=cap, tau=wl.tau, **kw)
     elif wl.mode == "global":
         k = wl.pair_count(wl.keep_num)
-        layer = bsa.DfsLayer(s, order=wl.order, mode="global", k=k, kcap=s.nb)
+        layer = bsa.DfsLayer(s, mode="global", k=k, kcap=s.nb, **kw)
     elif wl.mode == "radial":
-        layer = bsa.DfsLayer(s, order=wl.order, mode="radial", radial_w0=wl.radial_w0,
-                             radial_lambda=wl.radial_lambda)
+        layer = bsa.DfsLayer(s, mode="radial", radial_w0=wl.radial_w0, radial_lambda=wl.radial_lambda, **kw)
     else:
-        layer = bsa.DfsLayer(s, order=wl.order, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
-                             lvsa_step=wl.lvsa_step, frame_exact=wl.frame_exact)
+        layer = bsa.DfsLayer(s, mode="lvsa", lvsa_T_per=wl.lvsa_T_per, lvsa_C=wl.lvsa_C,
+                             lvsa_step=wl.lvsa_step, frame_exact=wl.frame_exact, **kw)
     return layer, k, cap
 
 
@@ -329,6 +334,114 @@ def run_ours(args):
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(wl, qkv, kk, cap, budget_s=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# dO reorder, prep, mask bits, transpose, dQ pass, dK/dV pass, three scatters
+BWD_KERNELS_PER_STEP = 8
+
+
+def run_backward(args):
+    import torch
+    import synth
+    import block_sparse_attention_36_b200 as bsa
+    from block_sparse_attention_36_b200 import dfsattn
+
+    rank, world, local = dist_setup(args.gpus)
+    wl = synth.WORKLOADS[args.workload]
+    qkv = synth.workload_inputs(wl, seed=args.seed + rank)
+    q, k, v = (qkv[n].cuda() for n in ("q", "k", "v"))
+    layer, kk, cap = make_layer(bsa, wl, want_lse=True)
+    layer.forward(q, k, v)
+    g = torch.Generator().manual_seed(args.seed + 1000 + rank)
+    dout_h = (torch.randn((wl.B, wl.N, wl.nh, wl.D), generator=g) * 0.5).to(torch.bfloat16)
+    dout = dout_h.cuda()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        layer.backward(dout)
+    torch.cuda.synchronize()
+    assert dfsattn.dfs_get_error_flags(clear=True) == 0
+    kept_pairs = layer.kept_pairs()
+    flops_step = 10.0 * wl.D * kept_pairs
+    b = layer._bwd
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    s = layer.shape
+    for i in range(args.steps):
+        dfsattn.dfs_hilbert_perm(s, layer.order, layer.perm, layer.inv, 0, dout, None, None, b["dop"], None, None)
+        ev[i][0].record(stream)
+        dfsattn.dfs_sparse_attn_bwd(s, layer.qp, layer.kp, layer.vp, layer.op, b["dop"], layer.lse, layer.kv_idx,
+                                    layer.kv_cnt, layer.kcap, layer.scale, b["dqp"], b["dkp"], b["dvp"], b["ws"])
+        ev[i][1].record(stream)
+        for name in ("dqp", "dkp", "dvp"):
+            dfsattn.dfs_unperm(s, layer.perm, b[name], layer.out)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    ms_total_max = max_over_ranks(start.elapsed_time(stop), world)
+    bwd_ms = statistics.mean(a.elapsed_time(c) for a, c in ev)
+    flops_all = sum_over_ranks(flops_step * args.steps, world)
+
+    # end to end: dO from pinned host memory in, the three gradients out
+    dh = dout_h.pin_memory()
+    hg = [torch.empty_like(dout_h).pin_memory() for _ in range(3)]
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        dout.copy_(dh, non_blocking=True)
+        grads = layer.backward(dout)
+        for h, d in zip(hg, grads):
+            h.copy_(d, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dout.copy_(dh, non_blocking=True)
+        grads = layer.backward(dout)
+        for h, d in zip(hg, grads):
+            h.copy_(d, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    assert dfsattn.dfs_get_error_flags(clear=True) == 0
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops_step / (bwd_ms * 1e-3) / 1e12
+        ms_step = ms_total_max / args.steps
+        line = {
+            "metric": "block-sparse attention backward: kept-block TFLOP/s (10*D FLOP per kept pair) vs B200 bf16 TC peak",
+            "value": round(flops_all / (ms_total_max * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s (kept-block backward, whole step)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4), "bwd_ms_per_call": round(bwd_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded smooth Fourier field + noise, bf16; dO Gaussian)",
+            "config": {"workload": workload_config(wl, kk, cap) + ", backward", "kept_pairs_per_step": kept_pairs,
+                       "executed_flop_per_pair": 14 * wl.D,
+                       "l2": "inputs larger than L2 (Q, K, V, O, dO, dQ, dK, dV: 8 x %.1f MB)"
+                             % (wl.N * wl.nh * wl.D * 2 / 1e6),
+                       "parallelism": f"replicas x{world} (independent layer per GPU)"},
+            "roofline": {"kernel": "dfs_sparse_attn_bwd (prep, mask bits, transpose, dQ pass, dK/dV pass)",
+                         "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "peak_source": f"{src} bf16 burst", "traffic": None},
+            "e2e": {"value": round(sum_over_ranks(flops_step, world) / (e2e_ms * 1e-3) / 1e12, 3),
+                    "unit": "TFLOP/s (kept-block backward, whole step)", "ms_per_step": round(e2e_ms, 3),
+                    "h2d_bytes_per_step": int(dh.numel() * dh.element_size()),
+                    "d2h_bytes_per_step": int(3 * dh.numel() * dh.element_size())},
+            "gpu_launches": BWD_KERNELS_PER_STEP * args.steps,
+            "clocks": clk,
+        }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -516,11 +629,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="replay each step as a captured CUDA graph")
+    ap.add_argument("--backward", action="store_true", help="time the gradient pass (DfsLayer.backward)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.backward:
+        run_backward(args)
     else:
         run_ours(args)
 

@@ -24,6 +24,7 @@ extern "C" int dfs_get_error_flags(uint32_t* flags, int clear) {
   if ((st = dfs_detail_flags_score(&v, clear)) != DFS_OK) return st;
   if ((st = dfs_detail_flags_select(&v, clear)) != DFS_OK) return st;
   if ((st = dfs_detail_flags_attn(&v, clear)) != DFS_OK) return st;
+  if ((st = dfs_detail_flags_bwd(&v, clear)) != DFS_OK) return st;
   *flags = v;
   return DFS_OK;
 }

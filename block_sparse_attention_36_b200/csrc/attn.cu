@@ -31,14 +31,11 @@
 // Tensor memory: S_A | S_B | O_A | O_B (BLK, BLK, D, D fp32 columns).
 // Every mbarrier wait is bounded (DFS_FLAG_WAIT_TIMEOUT, early return);
 // copies and MMAs in flight are drained before tensor memory is released.
-#include <cuda.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "exp2_poly.cuh"
 #include "lvsa.cuh"
 #include "sm100_ptx.cuh"
+#include "tmap.cuh"
 
 // Every DFS_ATTN_EXP2_EMU-th pair of softmax exponentials is computed on the
 // FMA pipe (0: all on the special-function unit).
@@ -483,45 +480,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }
 
 // ------------------------------------------------------------------ host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// [BH, N, D] bf16 viewed as a 3-D tensor (D fastest); box = 64 x rows x 1.
-bool make_map(CUtensorMap* map, const void* base, long long N, int D, long long BH, int rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int D, int BLK, int EMU, bool FRAME>
 int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
                 const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t st,
                 FrameMask fm) {
   using C = Cfg<D, BLK>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qp, d.N, D, d.BH, kQRows) || !make_map(&mk, kp, d.N, D, d.BH, BLK) ||
-      !make_map(&mv, vp, d.N, D, d.BH, BLK))
+  if (!dfs::make_map_bf16(&mq, qp, d.N, D, d.BH, kQRows) || !dfs::make_map_bf16(&mk, kp, d.N, D, d.BH, BLK) ||
+      !dfs::make_map_bf16(&mv, vp, d.N, D, d.BH, BLK))
     return DFS_ERR_CUDA;
   const int max_list = min(kcap, d.nb);
   size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + 2 * (size_t)max_list * sizeof(int32_t);

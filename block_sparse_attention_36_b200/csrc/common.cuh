@@ -79,6 +79,9 @@ extern "C" int dfs_detail_flags_perm(uint32_t* v, int clear);
 extern "C" int dfs_detail_flags_score(uint32_t* v, int clear);
 extern "C" int dfs_detail_flags_select(uint32_t* v, int clear);
 extern "C" int dfs_detail_flags_attn(uint32_t* v, int clear);
+extern "C" int dfs_detail_flags_bwd(uint32_t* v, int clear);
+// Workspace bytes of dfs_sparse_attn_bwd (0 for an unsupported shape).
+extern "C" size_t dfs_detail_ws_attn_bwd(const dfs_shape* shape);
 
 #define DFS_DEFINE_FLAG_READER(NAME, SYMBOL)                                   \
   extern "C" int NAME(uint32_t* v, int clear) {                               \

@@ -188,6 +188,7 @@ DFS_DEFINE_FLAG_READER(dfs_detail_flags_score, g_score_flags)
 
 extern "C" size_t dfs_workspace_bytes(const dfs_shape* shape, int which) {
   dfs::Dims d;
+  if (which == DFS_WS_ATTN_BWD) return dfs_detail_ws_attn_bwd(shape);
   if (which != DFS_WS_BLOCK_SCORE) return 0;
   if (dfs::check_shape(shape, &d, true) != DFS_OK) return 0;
   return (size_t)2 * d.BH * d.nsb * d.D * sizeof(float);

@@ -32,6 +32,7 @@ DFS_SEL_LVSA = 2
 DFS_SEL_GLOBAL = 3
 DFS_SEL_RADIAL = 4
 DFS_WS_BLOCK_SCORE = 0
+DFS_WS_ATTN_BWD = 1
 
 DFS_FLAG_WAIT_TIMEOUT = 1
 DFS_FLAG_BAD_KV_INDEX = 2
@@ -48,7 +49,7 @@ MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_L
 EXPORTS = (
     "dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd", "dfs_unperm",
     "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version", "dfs_block_score_noalloc",
-    "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd",
+    "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd", "dfs_sparse_attn_bwd",
 )
 
 
@@ -76,6 +77,7 @@ def _load():
     lib.dfs_hilbert_perm_pooled.argtypes = [sp, I, P, P, I, P, P, P, P, P, P, P, S, P]
     lib.dfs_block_score_pooled.argtypes = [sp, F, P, P, S, P]
     lib.dfs_sparse_attn_lvsa_fwd.argtypes = [sp, P, P, P, P, P, I, F, ctypes.POINTER(_SelectParams), P, P, P]
+    lib.dfs_sparse_attn_bwd.argtypes = [sp, P, P, P, P, P, P, P, P, I, F, P, P, P, P, S, P]
     lib.dfs_sparse_attn_fwd.argtypes = [sp, P, P, P, P, P, I, F, P, P, P]
     lib.dfs_unperm.argtypes = [sp, P, P, P, P]
     lib.dfs_workspace_bytes.argtypes = [sp, I]
@@ -86,7 +88,8 @@ def _load():
     lib.dfs_version.argtypes = []
     for name in ("dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd",
                  "dfs_unperm", "dfs_get_error_flags", "dfs_version", "dfs_block_score_noalloc",
-                 "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd"):
+                 "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd",
+                 "dfs_sparse_attn_bwd"):
         getattr(lib, name).restype = I
     return lib
 
@@ -208,6 +211,15 @@ def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o
     _check("dfs_sparse_attn_fwd", LIB.dfs_sparse_attn_fwd(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
         _ptr(op), _ptr(lse), _stream(stream)))
+
+
+def dfs_sparse_attn_bwd(shape: Shape, qp, kp, vp, op, dop, lse, kv_idx, kv_cnt, kcap, scale, dqp, dkp, dvp, ws,
+                        stream=None):
+    sh = shape.c()
+    _check("dfs_sparse_attn_bwd", LIB.dfs_sparse_attn_bwd(
+        ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(op), _ptr(dop), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt),
+        int(kcap), float(scale), _ptr(dqp), _ptr(dkp), _ptr(dvp), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def dfs_sparse_attn_lvsa_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, params, op, lse=None,

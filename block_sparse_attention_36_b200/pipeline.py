@@ -62,6 +62,7 @@ class DfsLayer:
             self.scores = None
             self.ws = None
         self._index_built = False
+        self._bwd = None
         # the fused reorder + pooling needs nh * D / 8 <= 512
         self.fused_pool = s.nh * s.D // 8 <= 512
 
@@ -143,6 +144,36 @@ class DfsLayer:
         with torch.cuda.graph(graph):
             self.forward(q, k, v, refresh_mask)
         return graph
+
+    def backward(self, dout, stream=None):
+        """Gradients of the last forward: dout is dL/dout, bf16 [B, N, nh, D]
+        in raster order (the layout of ``out``). Returns (dq, dk, dv) in the
+        same raster layout. Needs ``want_lse=True`` (the backward reads the
+        forward's log-sum-exp) and blk = 128; frame-exact LVSA has no
+        backward."""
+        if self.lse is None:
+            raise ValueError("backward needs the forward's lse: build the layer with want_lse=True")
+        if self.frame_exact:
+            raise ValueError("frame-exact LVSA attention has no backward")
+        s = self.shape
+        if self._bwd is None:
+            dev = self.qp.device
+            nbytes = lib.dfs_workspace_bytes(s, lib.DFS_WS_ATTN_BWD)
+            self._bwd = {
+                "ws": torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev),
+                "dop": torch.empty_like(self.qp), "dqp": torch.empty_like(self.qp),
+                "dkp": torch.empty_like(self.qp), "dvp": torch.empty_like(self.qp),
+            }
+        b = self._bwd
+        lib.dfs_hilbert_perm(s, self.order, self.perm, self.inv, 0, dout, None, None, b["dop"], None, None, stream)
+        lib.dfs_sparse_attn_bwd(s, self.qp, self.kp, self.vp, self.op, b["dop"], self.lse, self.kv_idx,
+                                self.kv_cnt, self.kcap, self.scale, b["dqp"], b["dkp"], b["dvp"], b["ws"], stream)
+        outs = []
+        for name in ("dqp", "dkp", "dvp"):
+            g = torch.empty((s.B, s.N, s.nh, s.D), dtype=torch.bfloat16, device=self.qp.device)
+            lib.dfs_unperm(s, self.perm, b[name], g, stream)
+            outs.append(g)
+        return tuple(outs)
 
     def kept_pairs(self):
         """Valid (query, key) token pairs the kept blocks cover (for FLOP counts)."""

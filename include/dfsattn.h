@@ -64,7 +64,7 @@ typedef struct {
 
 enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1, DFS_ORDER_TILE2D = 2, DFS_ORDER_TILE3D = 3 };
 enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2, DFS_SEL_GLOBAL = 3, DFS_SEL_RADIAL = 4 };
-enum { DFS_WS_BLOCK_SCORE = 0 };
+enum { DFS_WS_BLOCK_SCORE = 0, DFS_WS_ATTN_BWD = 1 };
 
 /* Device error word bits (dfs_get_error_flags). */
 enum {
@@ -238,6 +238,30 @@ int dfs_sparse_attn_fwd(const dfs_shape *shape, const void *qp, const void *kp, 
 int dfs_sparse_attn_lvsa_fwd(const dfs_shape *shape, const void *qp, const void *kp, const void *vp,
                              const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
                              const dfs_select_params *lvsa, void *op, float *lse, dfs_stream_t stream);
+
+/* dfs_sparse_attn_bwd -- gradients of dfs_sparse_attn_fwd over the same
+ * kept lists, as training through block attention needs them (VMoBA:
+ * Mixture of Block Attention for Video Diffusion Models, abstract: training
+ * speed-ups of the block attention).
+ *
+ * For a loss L with dL/dO = dop, and P = exp(scale q.k - lse) over the kept
+ * keys of each query's block, dP = dO V^T, Delta_q = dO_q . O_q,
+ * dS = P (dP - Delta):
+ *   dqp = scale dS K,  dkp = scale dS^T Q,  dvp = P^T dO
+ * qp, kp, vp, op, dop, dqp, dkp, dvp: bf16 [B, nh, N, D] (curve order);
+ * op and lse (fp32 [B, nh, N], natural log) are the forward's outputs for
+ * the same lists and scale. Lists must not repeat a block (as produced by
+ * dfs_select_mask). P and dS are rounded to bf16 for the tensor-core
+ * products, accumulation is fp32, the sums run in a fixed order (the
+ * result is deterministic). blk must be 128 (D 64 or 128), nb <= 8192.
+ * Workspace: dfs_workspace_bytes(shape, DFS_WS_ATTN_BWD) bytes, 256-byte
+ * aligned, owned by the caller and not read before it is written (the
+ * per-row constants and the transposed lists). Invalid list entries are
+ * skipped and set DFS_FLAG_BAD_KV_INDEX.                                   */
+int dfs_sparse_attn_bwd(const dfs_shape *shape, const void *qp, const void *kp, const void *vp,
+                        const void *op, const void *dop, const float *lse, const int32_t *kv_idx,
+                        const int32_t *kv_cnt, int kcap, float scale, void *dqp, void *dkp, void *dvp,
+                        void *ws, size_t ws_bytes, dfs_stream_t stream);
 
 /* dfs_unperm -- inverse reorder: o[b, perm[i], h, :] = op[b, h, i, :],
  * op bf16 [B, nh, N, D] (curve order) -> o bf16 [B, N, nh, D] (raster).   */
