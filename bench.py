@@ -48,8 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch from one ncu capture
 # (profiles/attn_fwd_<workload>.md), valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
-ATTN_TRAFFIC = {"wan_1p3b_layer": (297_875_968 + 84_863_488, "fe92b8f843351e08")}
-ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh")
+ATTN_TRAFFIC = {"wan_1p3b_layer": (298_639_872 + 82_235_136, "634b90f88875f78a")}
+ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 
 def attn_sources_hash():

@@ -386,26 +386,42 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int b = j & 1;
-      if (!mbar_wait_bounded(&bars->s_full[b], (uint32_t)((j >> 1) & 1), abort_flag, kWaitLimit) ||
-          !mbar_wait_bounded(&bars->dp_full, (uint32_t)(j & 1), abort_flag, kWaitLimit)) {
+      // P = 2^(S scale log2 e - lse log2 e) as soon as S(j) is there (it
+      // overlaps dP(j)), then dS = P (dP - Delta) once dP(j) is.
+      if (!mbar_wait_bounded(&bars->s_full[b], (uint32_t)((j >> 1) & 1), abort_flag, kWaitLimit)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + (b ? C::kS1 : C::kS0) + 64 * g;
       const uint32_t p_addr = tmem + lane_base + C::kDP + 64 * g;
+      float pv[64];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t sr[32], pr[32], out[16];
+        uint32_t sr[32];
         tmem_ld32(s_addr + 32 * c, sr);
-        tmem_ld32(p_addr + 32 * c, pr);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sc2, nl2);
-          const float2 p = make_float2(ex2(x.x), ex2(x.y));
+          pv[32 * c + 2 * e] = ex2(x.x);
+          pv[32 * c + 2 * e + 1] = ex2(x.y);
+        }
+      }
+      if (!mbar_wait_bounded(&bars->dp_full, (uint32_t)(j & 1), abort_flag, kWaitLimit)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pr[32], out[16];
+        tmem_ld32(p_addr + 32 * c, pr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
           const float2 t = __fadd2_rn(make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])), nd2);
-          const float2 ds = __fmul2_rn(p, t);
+          const float2 ds = __fmul2_rn(make_float2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]), t);
           out[e] = pack_bf16x2(ds.x, ds.y);
         }
         // columns 64g + 16c .. +15: fp32 S columns this thread already read
@@ -446,14 +462,20 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 struct __align__(8) BarsKV {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
-  uint64_t st_full, dpt_full, p_ready, kv_final, mma_done;
+  uint64_t st_full, dpt_full, p_ready, ds_ready, kv_final, mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int n_q;
 };
 
-// Per query block i of the transposed list: S^T(i), dP^T(i) -> [P^T, dS^T
-// ready] -> dV += P^T dO, dK += dS^T Q -> release the Q/dO stage.
+// Per query block i of the transposed list the P/dS warps run two phases:
+// A forms P^T(i) from S^T(i) (the exponentials) and hands it to dV(i);
+// B forms dS^T(i) once dP^T(i) is there and hands it to dK(i). MMA order:
+// S^T(0) dP^T(0), then per i: [P^T(i)] dV(i) S^T(i+1) [dS^T(i)] dK(i)
+// dP^T(i+1). S^T(i+1) reuses the columns of P^T(i) after dV(i) and
+// dP^T(i+1) those of dS^T(i) after dK(i) (in-order MMAs), so phase A of
+// i+1 overlaps dK(i) and dP^T(i+1), and phase B of i overlaps dV(i) and
+// S^T(i+1).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -480,6 +502,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->dpt_full, 1);
     mbar_init(&bars->p_ready, 8);
+    mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->kv_final, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
@@ -550,21 +573,40 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint64_t st_k = desc_sw128(smem_addr(smem + C::kStageOff), 16, 1024);
     const uint64_t st_mn = desc_sw128(smem_addr(smem + C::kStageOff), kBlk * 128, 1024);
     bool ok = true;
-    if (n > 0) ok = mbar_wait_bounded(&bars->kv_full, 0, abort_flag, kWaitLimit);
+    auto q_off = [](int i) { return (uint64_t)(((i & 1) * C::kStageBytes) >> 4); };
+    auto do_off = [](int i) { return (uint64_t)(((i & 1) * C::kStageBytes + C::kTile) >> 4); };
+    if (n > 0) {
+      ok = mbar_wait_bounded(&bars->kv_full, 0, abort_flag, kWaitLimit) &&
+           mbar_wait_bounded(&bars->q_full[0], 0, abort_flag, kWaitLimit);
+      if (ok) {
+        issue_nt<D>(tmem + C::kST, dk_k, st_k + q_off(0));     // S^T = K Q^T
+        mma_commit_warp(&bars->st_full);
+        issue_nt<D>(tmem + C::kDPT, dv_k, st_k + do_off(0));   // dP^T = V dO^T
+        mma_commit_warp(&bars->dpt_full);
+      }
+    }
     for (int i = 0; i < n && ok; ++i) {
-      const int st = i & 1;
-      if (!mbar_wait_bounded(&bars->q_full[st], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-      const uint64_t q_off = (uint64_t)((st * C::kStageBytes) >> 4);
-      const uint64_t do_off = (uint64_t)((st * C::kStageBytes + C::kTile) >> 4);
-      issue_nt<D>(tmem + C::kST, dk_k, st_k + q_off);      // S^T = K Q^T
-      mma_commit_warp(&bars->st_full);
-      issue_nt<D>(tmem + C::kDPT, dv_k, st_k + do_off);    // dP^T = V dO^T
-      mma_commit_warp(&bars->dpt_full);
+      // P^T(i) and dS^T(i) are written with tcgen05.st by other threads:
+      // order the MMAs that read them after their arrivals.
       if (!mbar_wait_bounded(&bars->p_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       tc_fence_after();
-      issue_tn<D>(tmem + C::kDV, tmem + C::kST, st_mn + do_off, i > 0);    // dV += P^T dO
-      issue_tn<D>(tmem + C::kDK, tmem + C::kDPT, st_mn + q_off, i > 0);    // dK += dS^T Q
-      mma_commit_warp(&bars->q_empty[st]);
+      issue_tn<D>(tmem + C::kDV, tmem + C::kST, st_mn + do_off(i), i > 0);    // dV += P^T dO
+      if (i + 1 < n) {
+        if (!mbar_wait_bounded(&bars->q_full[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1), abort_flag, kWaitLimit)) {
+          ok = false;
+          break;
+        }
+        issue_nt<D>(tmem + C::kST, dk_k, st_k + q_off(i + 1));
+        mma_commit_warp(&bars->st_full);
+      }
+      if (!mbar_wait_bounded(&bars->ds_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+      tc_fence_after();
+      issue_tn<D>(tmem + C::kDK, tmem + C::kDPT, st_mn + q_off(i), i > 0);    // dK += dS^T Q
+      mma_commit_warp(&bars->q_empty[i & 1]);
+      if (i + 1 < n) {
+        issue_nt<D>(tmem + C::kDPT, dv_k, st_k + do_off(i + 1));
+        mma_commit_warp(&bars->dpt_full);
+      }
     }
     if (ok && n > 0) mma_commit_warp(&bars->kv_final);
     mma_commit_warp(&bars->mma_done);
@@ -582,7 +624,6 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int st = i & 1;
       // q_full: the stage's -lse and -Delta rows, written by the bulk copy
       if (!mbar_wait_bounded(&bars->st_full, (uint32_t)(i & 1), abort_flag, kWaitLimit) ||
-          !mbar_wait_bounded(&bars->dpt_full, (uint32_t)(i & 1), abort_flag, kWaitLimit) ||
           !mbar_wait_bounded(&bars->q_full[st], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimit)) {
         ok = false;
         break;
@@ -592,31 +633,53 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const float* nd = nl + kBlk;
       const uint32_t s_addr = tmem + lane_base + C::kST + 64 * g;
       const uint32_t p_addr = tmem + lane_base + C::kDPT + 64 * g;
+      // phase A: P^T = 2^(S^T scale log2 e - lse log2 e), kept in fp32 for phase B
+      float pv[64];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t sr[32], pr[32], po[16], so[16];
+        uint32_t sr[32], po[16];
         tmem_ld32(s_addr + 32 * c, sr);
-        tmem_ld32(p_addr + 32 * c, pr);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int q = 64 * g + 32 * c + 2 * e;
           const float2 nl2 = *reinterpret_cast<const float2*>(nl + q);
-          const float2 nd2 = *reinterpret_cast<const float2*>(nd + q);
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sc2, nl2);
-          const float2 p = make_float2(ex2(x.x), ex2(x.y));
-          const float2 t = __fadd2_rn(make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])), nd2);
-          const float2 ds = __fmul2_rn(p, t);
-          po[e] = pack_bf16x2(p.x, p.y);
-          so[e] = pack_bf16x2(ds.x, ds.y);
+          pv[32 * c + 2 * e] = ex2(x.x);
+          pv[32 * c + 2 * e + 1] = ex2(x.y);
+          po[e] = pack_bf16x2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]);
         }
         tmem_st16(s_addr + 16 * c, po);
-        tmem_st16(p_addr + 16 * c, so);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
+      // phase B: dS^T = P^T (dP^T - Delta)
+      if (!mbar_wait_bounded(&bars->dpt_full, (uint32_t)(i & 1), abort_flag, kWaitLimit)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pr[32], so[16];
+        tmem_ld32(p_addr + 32 * c, pr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q = 64 * g + 32 * c + 2 * e;
+          const float2 nd2 = *reinterpret_cast<const float2*>(nd + q);
+          const float2 t = __fadd2_rn(make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])), nd2);
+          const float2 ds = __fmul2_rn(make_float2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]), t);
+          so[e] = pack_bf16x2(ds.x, ds.y);
+        }
+        tmem_st16(p_addr + 16 * c, so);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_ready);
     }
     if (ok && n > 0) ok = mbar_wait_bounded(&bars->kv_final, 0, abort_flag, kWaitLimit);
     tc_fence_after();
