@@ -8,7 +8,8 @@
 //   dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO.
 // Two deterministic passes (no atomics; every sum runs in a fixed order):
 //   attn_bwd_dq_kernel    one CTA per query block, over its kept list:
-//                         S = Q K^T, dP = dO V^T, dS, dQ += dS K.
+//                         S = Q K^T, dP = dO V^T, dS, dQ += dS K, with Q
+//                         and dO held in tensor memory.
 //   attn_bwd_dkdv_kernel  one CTA per key block, over the query blocks that
 //                         keep it (the transposed lists, ascending):
 //                         S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
@@ -40,7 +41,7 @@ constexpr long long kWaitLimit = 4000000000ll;
 constexpr long long kDrainLimit = 2000000000ll;
 constexpr int kThreads = 384;
 constexpr int kBlk = 128;      // block size = MMA M = N of the score products
-constexpr int kRing = 4;       // K/V ring stages of the dQ pass
+constexpr int kRing = 6;       // K/V ring stages of the dQ pass
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -48,10 +49,8 @@ template <int D>
 struct Bw {
   static constexpr int kChunks = D / 64;          // 128-byte column slabs per row
   static constexpr int kTile = kBlk * D * 2;      // one 128-row tile
-  // dQ pass shared memory
-  static constexpr int kQOff = 0;
-  static constexpr int kDOOff = kTile;
-  static constexpr int kRingOff = 2 * kTile;
+  // dQ pass shared memory: the K/V ring only
+  static constexpr int kRingOff = 0;
   static constexpr int kQBarOff = kRingOff + kRing * kTile;
   // dK/dV pass shared memory: K, V, then two stages of
   // {Q, dO, -lse log2 e [128], -Delta [128]}
@@ -61,7 +60,7 @@ struct Bw {
   static constexpr int kStageBytes = 2 * kTile + 1024;
   static constexpr int kKVBarOff = kStageOff + 2 * kStageBytes;
   // tensor memory columns
-  static constexpr int kS0 = 0, kS1 = 128, kDP = 256, kDQ = 384;      // dQ pass
+  static constexpr int kS = 0, kDP = 128, kDQ = 256, kQT = 256 + D, kDOT = 256 + D + D / 2;  // dQ pass
   static constexpr int kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D;  // dK/dV pass
 };
 
@@ -218,23 +217,38 @@ bwd_transpose_kernel(const uint32_t* __restrict__ bits, int nb, int nw, long lon
 
 // ------------------------------------------------------------ dQ pass
 struct __align__(8) BarsQ {
-  uint64_t q_full;
+  uint64_t qt_ready;
   uint64_t kv_full[kRing], kv_empty[kRing];
-  uint64_t s_full[2], dp_full, ds_ready, dq_final, mma_done;
+  uint64_t s_full, s_free, dp_full, ds_ready, dq_final, mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int n_kv;
 };
 
-// Tiles of the ring in load (= first use) order: K(0), V(0), K(1), V(1), ...
-// (tile u: K(u/2) for even u, V(u/2) for odd u). MMA order: S(0) dP(0) S(1),
-// then per kept block j: [dS(j) ready] dP(j+1), dQ += dS(j) K(j), S(j+2).
-// S is double-buffered: S(j+2) reuses S(j)'s columns after dQ(j) read dS(j)
-// there (tcgen05 MMAs of one thread run in order).
+// S = Q K^T or dP = dO V^T with the 128 x D left operand resident in tensor
+// memory (two bf16 per column, D/2 columns) and K or V a K-major tile.
+template <int D>
+__device__ __forceinline__ void issue_ts_nt(uint32_t d_tmem, uint32_t a_tmem, uint64_t db) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBlk, kBlk, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t off = (uint64_t)(((kk >> 2) * (kBlk * 128) + (kk & 3) * 32) >> 4);
+    mma_ts_warp(d_tmem, a_tmem + kk * 8, db + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Q and dO of the query block live in tensor memory for the whole CTA
+// (written once by the dS warps), so both score products read only K or V
+// from shared memory. Ring tiles in load (= first use) order: K(0), V(0),
+// K(1), V(1), ... (tile u: K(u/2) for even u, V(u/2) for odd u). MMA order:
+// S(0) dP(0), then per kept block j: [S(j) read] S(j+1), [dS(j) written
+// over dP(j)] dQ += dS(j) K(j), dP(j+1). S(j+1) therefore runs while the
+// exponentials of block j are formed, and dQ(j), dP(j+1) while those of
+// block j+1 are.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __nv_bfloat16* __restrict__ qp, const __nv_bfloat16* __restrict__ dop,
                    const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt, int kcap, int N, int nb,
                    float scale, float scale_log2, const float* __restrict__ nlse, const float* __restrict__ ndelta,
                    __nv_bfloat16* __restrict__ dq, int max_list) {
@@ -248,13 +262,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->qt_ready, 8);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 8);
     mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->dq_final, 1);
@@ -290,18 +304,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tensor_map(&tm_q);
       prefetch_tensor_map(&tm_k);
       prefetch_tensor_map(&tm_v);
-      prefetch_tensor_map(&tm_do);
-    }
-    if (n > 0) {
-      mbar_arrive_expect_tx_warp(&bars->q_full, 2 * C::kTile);
-#pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d_warp(smem + C::kQOff + c * (kBlk * 128), &tm_q, &bars->q_full, c * 64, I * kBlk, bh);
-        tma_load_3d_warp(smem + C::kDOOff + c * (kBlk * 128), &tm_do, &bars->q_full, c * 64, I * kBlk, bh);
-      }
     }
     int u = 0;
     for (; u < 2 * n; ++u) {
@@ -319,11 +323,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // so only the last kRing loads can still be in flight.
     for (int w = max(0, u - kRing); w < u; ++w)
       mbar_wait_timed(&bars->kv_full[w % kRing], (uint32_t)((w / kRing) & 1), kDrainLimit);
-    if (n > 0) mbar_wait_timed(&bars->q_full, 0, kDrainLimit);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    const uint64_t dq_k = desc_sw128(smem_addr(smem + C::kQOff), 16, 1024);
-    const uint64_t ddo_k = desc_sw128(smem_addr(smem + C::kDOOff), 16, 1024);
     const uint64_t ring_k = desc_sw128(smem_addr(smem + C::kRingOff), 16, 1024);
     const uint64_t ring_mn = desc_sw128(smem_addr(smem + C::kRingOff), kBlk * 128, 1024);
     auto stage_off = [](int u) { return (uint64_t)(((u % kRing) * C::kTile) >> 4); };
@@ -332,41 +333,40 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     };
     bool ok = true;
     if (n > 0) {
-      ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, kWaitLimit);
+      // Q and dO were stored into tensor memory with tcgen05.st.
+      ok = mbar_wait_bounded(&bars->qt_ready, 0, abort_flag, kWaitLimit);
+      tc_fence_after();
       if (ok && (ok = wait_tile(0))) {
-        issue_nt<D>(tmem + C::kS0, dq_k, ring_k + stage_off(0));
-        mma_commit_warp(&bars->s_full[0]);
+        issue_ts_nt<D>(tmem + C::kS, tmem + C::kQT, ring_k + stage_off(0));
+        mma_commit_warp(&bars->s_full);
       }
       if (ok && (ok = wait_tile(1))) {
-        issue_nt<D>(tmem + C::kDP, ddo_k, ring_k + stage_off(1));
+        issue_ts_nt<D>(tmem + C::kDP, tmem + C::kDOT, ring_k + stage_off(1));
         mma_commit_warp(&bars->dp_full);
         mma_commit_warp(&bars->kv_empty[1 % kRing]);
       }
-      if (ok && n > 1 && (ok = wait_tile(2))) {
-        issue_nt<D>(tmem + C::kS1, dq_k, ring_k + stage_off(2));
-        mma_commit_warp(&bars->s_full[1]);
-      }
     }
     for (int j = 0; j < n && ok; ++j) {
-      // dS(j) was written by the softmax warps with tcgen05.st: order the
-      // MMAs that read it (and overwrite dP) after their arrival.
+      if (j + 1 < n) {
+        // S(j) has been read into registers: S(j+1) may overwrite it.
+        if (!mbar_wait_bounded(&bars->s_free, (uint32_t)(j & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+        tc_fence_after();
+        const int u = 2 * (j + 1);       // K(j+1)
+        if (!wait_tile(u)) { ok = false; break; }
+        issue_ts_nt<D>(tmem + C::kS, tmem + C::kQT, ring_k + stage_off(u));
+        mma_commit_warp(&bars->s_full);
+      }
+      // dS(j) was written over dP(j) with tcgen05.st by the dS warps.
       if (!mbar_wait_bounded(&bars->ds_ready, (uint32_t)(j & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       tc_fence_after();
+      issue_tn<D>(tmem + C::kDQ, tmem + C::kDP, ring_mn + stage_off(2 * j), j > 0);   // K(j), MN-major
+      mma_commit_warp(&bars->kv_empty[(2 * j) % kRing]);
       if (j + 1 < n) {
         const int u = 2 * (j + 1) + 1;   // V(j+1)
         if (!wait_tile(u)) { ok = false; break; }
-        issue_nt<D>(tmem + C::kDP, ddo_k, ring_k + stage_off(u));
+        issue_ts_nt<D>(tmem + C::kDP, tmem + C::kDOT, ring_k + stage_off(u));
         mma_commit_warp(&bars->dp_full);
         mma_commit_warp(&bars->kv_empty[u % kRing]);
-      }
-      const uint32_t s_buf = tmem + ((j & 1) ? C::kS1 : C::kS0);
-      issue_tn<D>(tmem + C::kDQ, s_buf, ring_mn + stage_off(2 * j), j > 0);   // K(j), MN-major
-      mma_commit_warp(&bars->kv_empty[(2 * j) % kRing]);
-      if (j + 2 < n) {
-        const int u = 2 * (j + 2);       // K(j+2)
-        if (!wait_tile(u)) { ok = false; break; }
-        issue_nt<D>(s_buf, dq_k, ring_k + stage_off(u));
-        mma_commit_warp(&bars->s_full[j & 1]);
       }
     }
     if (ok && n > 0) mma_commit_warp(&bars->dq_final);
@@ -380,32 +380,66 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int sub = warp & 3;                       // TMEM lane quarter
     const int r = sub * 32 + lane;                  // query row in the block
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
+    const long long qrow = (long long)I * kBlk + r;
+    {
+      // this row's half of Q and dO into tensor memory (zeros past N)
+      constexpr int kHalf = D / 2;                  // elements per warpgroup
+      const long long off = ((long long)bh * N + qrow) * D + kHalf * g;
+      const bool in = qrow < N;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint4* src = reinterpret_cast<const uint4*>((t == 0 ? qp : dop) + off);
+        const uint32_t col = tmem + lane_base + (t == 0 ? C::kQT : C::kDOT) + (kHalf / 2) * g;
+        if (kHalf == 64) {
+          uint32_t w[32];
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = in ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+          }
+          tmem_st32(col, w);
+        } else {
+          uint32_t w[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 x = in ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+          }
+          tmem_st16(col, w);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qt_ready);
+    }
     const long long prow = ((long long)bh * nb + I) * kBlk + r;
     const float nl = nlse[prow], nd = ndelta[prow];
     const float2 sc2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(nl, nl), nd2 = make_float2(nd, nd);
+    const uint32_t s_addr = tmem + lane_base + C::kS + 64 * g;
+    const uint32_t p_addr = tmem + lane_base + C::kDP + 64 * g;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      // P = 2^(S scale log2 e - lse log2 e) as soon as S(j) is there (it
-      // overlaps dP(j)), then dS = P (dP - Delta) once dP(j) is.
-      if (!mbar_wait_bounded(&bars->s_full[b], (uint32_t)((j >> 1) & 1), abort_flag, kWaitLimit)) {
+      // S(j) into registers, release it, then P = 2^(S scale log2 e - lse log2 e)
+      if (!mbar_wait_bounded(&bars->s_full, (uint32_t)(j & 1), abort_flag, kWaitLimit)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_base + (b ? C::kS1 : C::kS0) + 64 * g;
-      const uint32_t p_addr = tmem + lane_base + C::kDP + 64 * g;
       float pv[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(s_addr + 32 * c, sr);
+      {
+        uint32_t sr[64];
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 32; ++e) {
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sc2, nl2);
-          pv[32 * c + 2 * e] = ex2(x.x);
-          pv[32 * c + 2 * e + 1] = ex2(x.y);
+          pv[2 * e] = ex2(x.x);
+          pv[2 * e + 1] = ex2(x.y);
         }
       }
       if (!mbar_wait_bounded(&bars->dp_full, (uint32_t)(j & 1), abort_flag, kWaitLimit)) {
@@ -424,8 +458,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const float2 ds = __fmul2_rn(make_float2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]), t);
           out[e] = pack_bf16x2(ds.x, ds.y);
         }
-        // columns 64g + 16c .. +15: fp32 S columns this thread already read
-        tmem_st16(s_addr + 16 * c, out);
+        // columns 64g + 16c .. +15 of dP: fp32 columns this thread already read
+        tmem_st16(p_addr + 16 * c, out);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -434,7 +468,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (ok && n > 0) ok = mbar_wait_bounded(&bars->dq_final, 0, abort_flag, kWaitLimit);
     tc_fence_after();
-    const long long qrow = (long long)I * kBlk + r;
     const bool store = ok && qrow < N;
     __nv_bfloat16* orow = dq + ((long long)bh * N + qrow) * D + (D / 2) * g;
 #pragma unroll
@@ -774,8 +807,9 @@ int launch_bwd(const dfs::Dims& d, const void* qp, const void* kp, const void* v
                                                                                       nw, w.bits);
   bwd_transpose_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, cs>>>(w.bits, nb, nw, rows, w.q_idx, w.q_cnt);
   const dim3 grid((unsigned)nb, (unsigned)d.BH);
-  attn_bwd_dq_kernel<D><<<grid, kThreads, smem_q, cs>>>(mq, mk, mv, mdo, kv_idx, kv_cnt, kcap, (int)d.N, nb, scale,
-                                                         scale_log2, w.nlse, w.ndelta, (__nv_bfloat16*)dqp, max_list);
+  attn_bwd_dq_kernel<D><<<grid, kThreads, smem_q, cs>>>(mk, mv, (const __nv_bfloat16*)qp, (const __nv_bfloat16*)dop,
+                                                         kv_idx, kv_cnt, kcap, (int)d.N, nb, scale, scale_log2,
+                                                         w.nlse, w.ndelta, (__nv_bfloat16*)dqp, max_list);
   attn_bwd_dkdv_kernel<D><<<grid, kThreads, smem_kv, cs>>>(mq, mk, mv, mdo, w.q_idx, w.q_cnt, (int)d.N, nb, scale,
                                                             scale_log2, w.nlse, w.ndelta, (__nv_bfloat16*)dkp,
                                                             (__nv_bfloat16*)dvp);
