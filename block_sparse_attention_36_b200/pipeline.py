@@ -63,6 +63,7 @@ class DfsLayer:
             self.ws = None
         self._index_built = False
         self._bwd = None
+        self._pipe = None
         # the fused reorder + pooling needs nh * D / 8 <= 512
         self.fused_pool = s.nh * s.D // 8 <= 512
 
@@ -90,9 +91,9 @@ class DfsLayer:
             lib.dfs_block_score(self.shape, self.qp, self.kp, self.scale, self.scores, self.ws, stream)
         lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
 
-    def attend(self, stream=None):
+    def attend(self, stream=None, out=None):
         self.attention(stream)
-        lib.dfs_unperm(self.shape, self.perm, self.op, self.out, stream)
+        lib.dfs_unperm(self.shape, self.perm, self.op, self.out if out is None else out, stream)
 
     def attention(self, stream=None):
         """The attention kernel alone (curve order, into ``op``)."""
@@ -122,11 +123,64 @@ class DfsLayer:
             if refresh_mask:
                 self.build_mask(stream)
 
-    def forward(self, q, k, v, refresh_mask=True, stream=None):
-        """q, k, v: bf16 [B, N, nh, D] on the device (raster order). Returns the output buffer."""
+    def forward(self, q, k, v, refresh_mask=True, stream=None, out=None):
+        """q, k, v: bf16 [B, N, nh, D] on the device (raster order). Returns
+        the output buffer (``out`` if given, else the layer's own)."""
         self.prepare(q, k, v, refresh_mask, stream)
-        self.attend(stream)
-        return self.out
+        self.attend(stream, out)
+        return self.out if out is None else out
+
+    def run_host_steps(self, host_inputs, host_outputs, refresh_mask=True):
+        """Runs one step per (q, k, v) of ``host_inputs`` (pinned host bf16
+        [B, N, nh, D]) and copies each result into the matching pinned host
+        tensor of ``host_outputs``. Steps are pipelined over three streams:
+        the host-to-device copy of step i+1 and the device-to-host copy of
+        step i-1 overlap the kernels of step i (two device input sets and two
+        output buffers, ordered by events). Enqueues the work after the
+        current stream's pending work and makes the current stream wait for
+        all of it; returns without synchronising."""
+        n = len(host_inputs)
+        if len(host_outputs) != n:
+            raise ValueError("one host output per step")
+        s = self.shape
+        dev = self.qp.device
+        if self._pipe is None:
+            shape = (s.B, s.N, s.nh, s.D)
+            self._pipe = {
+                "inp": [[torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3)] for _ in range(2)],
+                "out": [torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(2)],
+                "streams": [torch.cuda.Stream(device=dev) for _ in range(3)],
+            }
+        p = self._pipe
+        s_in, s_cmp, s_out = p["streams"]
+        start = torch.cuda.current_stream()
+        for st in (s_in, s_cmp, s_out):
+            st.wait_stream(start)
+        cmp_done = [None, None]
+        out_done = [None, None]
+        for i in range(n):
+            b = i & 1
+            inp, dout = p["inp"][b], p["out"][b]
+            with torch.cuda.stream(s_in):
+                if cmp_done[b] is not None:
+                    s_in.wait_event(cmp_done[b])       # step i-2 has read this input set
+                for d, h in zip(inp, host_inputs[i]):
+                    d.copy_(h, non_blocking=True)
+                in_ready = torch.cuda.Event()
+                in_ready.record(s_in)
+            s_cmp.wait_event(in_ready)
+            if out_done[b] is not None:
+                s_cmp.wait_event(out_done[b])          # step i-2's result has left this buffer
+            self.forward(inp[0], inp[1], inp[2], refresh_mask, stream=s_cmp, out=dout)
+            cmp_done[b] = torch.cuda.Event()
+            cmp_done[b].record(s_cmp)
+            s_out.wait_event(cmp_done[b])
+            with torch.cuda.stream(s_out):
+                host_outputs[i].copy_(dout, non_blocking=True)
+                out_done[b] = torch.cuda.Event()
+                out_done[b].record(s_out)
+        for st in (s_in, s_cmp, s_out):
+            start.wait_stream(st)
 
     def capture_graph(self, q, k, v, refresh_mask=True, warmup=2):
         """Record one whole step (prepare + attend) into a CUDA graph over the
