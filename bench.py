@@ -41,14 +41,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
-# fused gather + pooling (1 launch), score, select, attention, scatter; LVSA: 3 gathers, select, attention, scatter
-KERNELS_PER_STEP = {"topk": 5, "threshold": 5, "global": 5, "lvsa": 6, "radial": 6}
+# fused gather + pooling (1 launch), score, select, attention with the scatter fused in;
+# LVSA / log-radial: 3 gathers, select, attention (frame-exact LVSA: + a separate scatter)
+# (threshold and global add the work-order sort)
+KERNELS_PER_STEP = {"topk": 4, "threshold": 5, "global": 5, "lvsa": 5, "radial": 5}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per attention launch from one ncu capture
 # (profiles/attn_fwd_<workload>.md), valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
-ATTN_TRAFFIC = {"wan_1p3b_layer": (298_639_872 + 82_235_136, "634b90f88875f78a")}
+ATTN_TRAFFIC = {"wan_1p3b_layer": (298_673_152 + 82_699_520, "99ab3bb278d64954")}
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 
@@ -252,9 +254,8 @@ def run_ours(args):
             continue
         layer.prepare(q, k, v)
         ev_attn[i][0].record(stream)
-        layer.attention()
+        layer.attend()          # attention with the inverse reorder fused into its epilogue
         ev_attn[i][1].record(stream)
-        dfsattn.dfs_unperm(layer.shape, layer.perm, layer.op, layer.out)
     stop.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -264,7 +265,7 @@ def run_ours(args):
         # attention-kernel time from eager launches (events cannot sit inside the graph replay)
         for i in range(args.steps):
             ev_attn[i][0].record(stream)
-            layer.attention()
+            layer.attend()
             ev_attn[i][1].record(stream)
         torch.cuda.synchronize()
         del graph
@@ -328,7 +329,7 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (3 x %.1f MB of Q/K/V per step)" % (wl.N * wl.nh * wl.D * 2 / 1e6),
                        "parallelism": f"replicas x{world} (independent layer per GPU)",
                        "launch": "CUDA graph replay" if args.graph else "eager launches"},
-            "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(achieved, 2),
+            "roofline": {"kernel": "attn_fwd_kernel (inverse reorder fused into the epilogue)", "bound": "tensor", "achieved": round(achieved, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                          "peak_source": f"{src} bf16 burst", "traffic": traffic},
             "e2e": {"value": round(e2e_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s (kept-block, whole step)",
@@ -337,7 +338,7 @@ def run_ours(args):
                     "d2h_bytes_per_step": int(hq.numel() * hq.element_size()),
                     "api": "DfsLayer.run_host_steps (copies of neighbouring steps overlap the kernels)",
                     "serial_ms_per_step": round(serial_ms, 3)},
-            "gpu_launches": KERNELS_PER_STEP[wl.mode] * args.steps,
+            "gpu_launches": (KERNELS_PER_STEP[wl.mode] + (1 if wl.frame_exact else 0)) * args.steps,
             "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:

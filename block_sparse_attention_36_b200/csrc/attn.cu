@@ -111,6 +111,18 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
 struct FrameMask {
   int P, T, T_per, s0, C, nG;
 };
+// Output rows go to op in curve order, or, when perm is set, straight to
+// their raster place o[b, perm[i], h, :] (o: [B, N, nh, D]). When order is
+// set, CTA c takes the query rows (b * nh + h) * nb + I at order[2c] and
+// order[2c + 1] (rows = B * nh * nb entries) instead of blocks 2c, 2c + 1
+// of head blockIdx.y.
+struct OutMap {
+  const int32_t* perm;
+  int nh;
+  const int32_t* order;
+  long long rows;
+};
+
 constexpr int kFrameRows = 3;
 constexpr int kMaxFrames = 4096;
 __host__ __device__ constexpr int frame_words(int T) { return (T + 31) / 32; }
@@ -120,7 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ kv_idx,
                 const int32_t* __restrict__ kv_cnt, int kcap, int N, int nb, float scale_log2,
-                __nv_bfloat16* __restrict__ op, float* __restrict__ lse, int max_list, FrameMask fm) {
+                __nv_bfloat16* __restrict__ op, float* __restrict__ lse, int max_list, FrameMask fm,
+                OutMap om) {
   using C = Cfg<D, BLK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -128,8 +141,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   int32_t* lists = reinterpret_cast<int32_t*>(smem + C::kBarOff + sizeof(Barriers));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int I0 = 2 * blockIdx.x;  // slot A: I0, slot B: I0 + 1
+  // (head, query block) of each slot; an empty slot gets block nb
+  int bh0 = blockIdx.y, bh1 = blockIdx.y, I0 = 2 * blockIdx.x, I1 = 2 * blockIdx.x + 1;
+  if (om.order) {
+    const long long pos = 2LL * blockIdx.x;
+    const int r0 = om.order[pos];
+    const int r1 = pos + 1 < om.rows ? om.order[pos + 1] : -1;
+    bh0 = r0 / nb;
+    I0 = r0 - bh0 * nb;
+    bh1 = r1 >= 0 ? r1 / nb : 0;
+    I1 = r1 >= 0 ? r1 - bh1 * nb : nb;
+  }
+  auto slot_bh = [&](int x) { return x ? bh1 : bh0; };
+  auto slot_I = [&](int x) { return x ? I1 : I0; };   // frame-exact masking (no order): I1 = I0 + 1
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
@@ -150,11 +174,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 2 || warp == 3) {
     // Compact the slot's kept list into shared memory, dropping invalid indices.
     const int x = warp - 2;
-    const int I = I0 + x;
+    const int I = slot_I(x);
     int base = 0;
     bool bad = false;
     if (I < nb) {
-      const long long row_id = (long long)bh * nb + I;
+      const long long row_id = (long long)slot_bh(x) * nb + I;
       int cnt = kv_cnt[row_id];
       cnt = max(0, min(cnt, min(kcap, max_list)));
       const int32_t* src = kv_idx + row_id * (long long)kcap;
@@ -221,7 +245,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_arrive_expect_tx_warp(&bars->q_full[x], C::kQBytes);
         for (int c = 0; c < C::kChunks; ++c)
           tma_load_3d_warp(smem + C::kQOff + x * C::kQBytes + c * (kQRows * 128), &tm_q, &bars->q_full[x], c * 64,
-                      (I0 + x) * BLK, bh);
+                           slot_I(x) * BLK, slot_bh(x));
       }
       // Same step order as the MMA issuer: step -1 loads K_A(0), K_B(0); step
       // j loads, per slot, V(j) and then K(j+1).
@@ -247,7 +271,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const CUtensorMap* map = kind == 0 ? &tm_v : &tm_k;
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d_warp(dst + c * (BLK * 128), map, &bars->kv_full[st], c * 64, J * BLK, bh);
+              tma_load_3d_warp(dst + c * (BLK * 128), map, &bars->kv_full[st], c * 64, J * BLK, slot_bh(x));
             ++t;
           }
           if (!ok) break;
@@ -316,7 +340,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else {
     // ------------------------------------------------------------ softmax
     const int x = warp < 8 ? 0 : 1;                 // slot
-    const int I = I0 + x;
+    const int I = slot_I(x);
+    const int bh = slot_bh(x);
     const int sub = warp & 3;                       // TMEM lane quarter of this warp
     const int r = sub * 32 + lane;                  // query row in the tile
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
@@ -444,7 +469,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const long long qrow = (long long)I * BLK + r;
     const bool store = ok && I < nb && r < BLK && qrow < N;
-    __nv_bfloat16* orow = op + ((long long)bh * N + qrow) * D;
+    __nv_bfloat16* orow;
+    if (om.perm) {
+      const int b = bh / om.nh, h = bh - b * om.nh;
+      const long long tok = (qrow < N) ? om.perm[qrow] : 0;
+      orow = op + (((long long)b * N + tok) * om.nh + h) * D;
+    } else {
+      orow = op + ((long long)bh * N + qrow) * D;
+    }
     const float inv_l = (nx > 0 && l > 0.f) ? 1.0f / l : 0.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -483,7 +515,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 template <int D, int BLK, int EMU, bool FRAME>
 int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
                 const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t st,
-                FrameMask fm) {
+                FrameMask fm, OutMap om) {
   using C = Cfg<D, BLK>;
   CUtensorMap mq, mk, mv;
   if (!dfs::make_map_bf16(&mq, qp, d.N, D, d.BH, kQRows) || !dfs::make_map_bf16(&mk, kp, d.N, D, d.BH, BLK) ||
@@ -501,10 +533,10 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, EMU, FRAME>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return DFS_ERR_CUDA;
-  dim3 grid((unsigned)((d.nb + 1) / 2), (unsigned)d.BH);
+  const dim3 grid = om.order ? dim3((unsigned)((d.BH * d.nb + 1) / 2), 1u) : dim3((unsigned)((d.nb + 1) / 2), (unsigned)d.BH);
   const float scale_log2 = scale * 1.4426950408889634f;
   attn_fwd_kernel<D, BLK, EMU, FRAME><<<grid, kThreads, smem, st>>>(
-      mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb, scale_log2, (__nv_bfloat16*)op, lse, max_list, fm);
+      mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb, scale_log2, (__nv_bfloat16*)op, lse, max_list, fm, om);
   return dfs::launch_status();
 }
 
@@ -529,15 +561,15 @@ int check_attn_args(const dfs_shape* shape, const void* qp, const void* kp, cons
 template <bool FRAME>
 int dispatch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* vp, const int32_t* kv_idx,
                   const int32_t* kv_cnt, int kcap, float scale, void* op, float* lse, cudaStream_t cs,
-                  FrameMask fm) {
+                  FrameMask fm, OutMap om) {
   constexpr int kEmu = DFS_ATTN_EXP2_EMU;
   if (d.D == 128 && d.blk == 128)
-    return launch_attn<128, 128, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
+    return launch_attn<128, 128, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm, om);
   if (d.D == 128 && d.blk == 64)
-    return launch_attn<128, 64, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
+    return launch_attn<128, 64, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm, om);
   if (d.D == 64 && d.blk == 128)
-    return launch_attn<64, 128, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
-  return launch_attn<64, 64, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm);
+    return launch_attn<64, 128, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm, om);
+  return launch_attn<64, 64, kEmu, FRAME>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, cs, fm, om);
 }
 
 }  // namespace
@@ -550,7 +582,24 @@ extern "C" int dfs_sparse_attn_fwd(const dfs_shape* shape, const void* qp, const
   if (st != DFS_OK) return st;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
   return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream,
-                              FrameMask{1, 1, 1, 0, 1, 0});
+                              FrameMask{1, 1, 1, 0, 1, 0}, OutMap{nullptr, 1, nullptr, 0});
+}
+
+extern "C" int dfs_sparse_attn_fwd_ex(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
+                                      const int32_t* kv_idx, const int32_t* kv_cnt, int kcap, float scale,
+                                      const dfs_attn_opts* opts, void* o, float* lse, dfs_stream_t stream) {
+  dfs::Dims d;
+  const int st = check_attn_args(shape, qp, kp, vp, kv_idx, kv_cnt, kcap, o, lse, &d);
+  if (st != DFS_OK) return st;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
+  OutMap om{nullptr, d.nh, nullptr, d.BH * d.nb};
+  if (opts) {
+    om.perm = opts->perm;
+    om.order = opts->order;
+  }
+  if (om.order && (d.BH * d.nb + 1) / 2 > 0x7fffffffLL) return DFS_ERR_UNSUPPORTED;
+  return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse, (cudaStream_t)stream,
+                              FrameMask{1, 1, 1, 0, 1, 0}, om);
 }
 
 extern "C" int dfs_sparse_attn_lvsa_fwd(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
@@ -570,5 +619,57 @@ extern "C" int dfs_sparse_attn_lvsa_fwd(const dfs_shape* shape, const void* qp, 
   fm.s0 = lvsa->lvsa_step % lvsa->lvsa_T_per;
   fm.C = lvsa->lvsa_C;
   fm.nG = (fm.s0 < d.T) ? (d.T - 1 - fm.s0) / fm.T_per + 1 : 0;
-  return dispatch_attn<true>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream, fm);
+  return dispatch_attn<true>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream, fm,
+                             OutMap{nullptr, 1, nullptr, 0});
+}
+
+namespace {
+
+// Counting sort of the query rows by kept count, descending, in one CTA:
+// shared-memory histogram, a scan from the largest count down, and a
+// scatter through per-count cursors (warp-aggregated, so rows of equal
+// count keep their order inside a warp's 32-row chunk).
+__global__ void __launch_bounds__(1024)
+attn_order_kernel(const int32_t* __restrict__ kv_cnt, long long rows, int kmax, int32_t* __restrict__ order) {
+  extern __shared__ int cursor[];   // kmax + 1 counters
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int c = tid; c <= kmax; c += blockDim.x) cursor[c] = 0;
+  __syncthreads();
+  for (long long r = tid; r < rows; r += blockDim.x) atomicAdd(&cursor[max(0, min(kv_cnt[r], kmax))], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int c = kmax; c >= 0; --c) {
+      const int h = cursor[c];
+      cursor[c] = run;
+      run += h;
+    }
+  }
+  __syncthreads();
+  for (long long r0 = (long long)(tid >> 5) * 32; r0 < rows; r0 += blockDim.x) {
+    const long long r = r0 + lane;
+    const bool in = r < rows;
+    const int c = in ? max(0, min(kv_cnt[r], kmax)) : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    const int leader = __ffs(peers) - 1;
+    int base = 0;
+    if (in && lane == leader) base = atomicAdd(&cursor[c], __popc(peers));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (in) order[base + __popc(peers & ((1u << lane) - 1u))] = (int32_t)r;
+  }
+}
+
+}  // namespace
+
+extern "C" int dfs_attn_order(const dfs_shape* shape, const int32_t* kv_cnt, int kcap, int32_t* order,
+                              dfs_stream_t stream) {
+  dfs::Dims d;
+  const int st = dfs::check_shape(shape, &d, false);
+  if (st != DFS_OK) return st;
+  if (!kv_cnt || !order || kcap < 1) return DFS_ERR_INVALID_ARG;
+  const int kmax = min(kcap, d.nb);
+  if (d.BH * d.nb >= (1LL << 31)) return DFS_ERR_UNSUPPORTED;
+  attn_order_kernel<<<1, 1024, (size_t)(kmax + 1) * sizeof(int), (cudaStream_t)stream>>>(kv_cnt, d.BH * d.nb, kmax,
+                                                                                          order);
+  return dfs::launch_status();
 }

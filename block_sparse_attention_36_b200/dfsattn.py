@@ -50,11 +50,16 @@ EXPORTS = (
     "dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd", "dfs_unperm",
     "dfs_workspace_bytes", "dfs_get_error_flags", "dfs_status_string", "dfs_version", "dfs_block_score_noalloc",
     "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd", "dfs_sparse_attn_bwd",
+    "dfs_sparse_attn_fwd_ex", "dfs_attn_order",
 )
 
 
 class _Shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "nh", "D", "T", "H", "W", "blk", "sb")]
+
+
+class _AttnOpts(ctypes.Structure):
+    _fields_ = [("perm", ctypes.c_void_p), ("order", ctypes.c_void_p)]
 
 
 class _SelectParams(ctypes.Structure):
@@ -78,6 +83,8 @@ def _load():
     lib.dfs_block_score_pooled.argtypes = [sp, F, P, P, S, P]
     lib.dfs_sparse_attn_lvsa_fwd.argtypes = [sp, P, P, P, P, P, I, F, ctypes.POINTER(_SelectParams), P, P, P]
     lib.dfs_sparse_attn_bwd.argtypes = [sp, P, P, P, P, P, P, P, P, I, F, P, P, P, P, S, P]
+    lib.dfs_sparse_attn_fwd_ex.argtypes = [sp, P, P, P, P, P, I, F, ctypes.POINTER(_AttnOpts), P, P, P]
+    lib.dfs_attn_order.argtypes = [sp, P, I, P, P]
     lib.dfs_sparse_attn_fwd.argtypes = [sp, P, P, P, P, P, I, F, P, P, P]
     lib.dfs_unperm.argtypes = [sp, P, P, P, P]
     lib.dfs_workspace_bytes.argtypes = [sp, I]
@@ -89,7 +96,7 @@ def _load():
     for name in ("dfs_hilbert_perm", "dfs_block_score", "dfs_select_mask", "dfs_sparse_attn_fwd",
                  "dfs_unperm", "dfs_get_error_flags", "dfs_version", "dfs_block_score_noalloc",
                  "dfs_hilbert_perm_pooled", "dfs_block_score_pooled", "dfs_sparse_attn_lvsa_fwd",
-                 "dfs_sparse_attn_bwd"):
+                 "dfs_sparse_attn_bwd", "dfs_sparse_attn_fwd_ex", "dfs_attn_order"):
         getattr(lib, name).restype = I
     return lib
 
@@ -211,6 +218,21 @@ def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o
     _check("dfs_sparse_attn_fwd", LIB.dfs_sparse_attn_fwd(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
         _ptr(op), _ptr(lse), _stream(stream)))
+
+
+def dfs_sparse_attn_fwd_ex(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse=None, perm=None,
+                           order=None, stream=None):
+    sh = shape.c()
+    opts = _AttnOpts(None if perm is None else perm.data_ptr(), None if order is None else order.data_ptr())
+    _check("dfs_sparse_attn_fwd_ex", LIB.dfs_sparse_attn_fwd_ex(
+        ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
+        ctypes.byref(opts), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def dfs_attn_order(shape: Shape, kv_cnt, kcap, order, stream=None):
+    sh = shape.c()
+    _check("dfs_attn_order", LIB.dfs_attn_order(ctypes.byref(sh), _ptr(kv_cnt), int(kcap), _ptr(order),
+                                                _stream(stream)))
 
 
 def dfs_sparse_attn_bwd(shape: Shape, qp, kp, vp, op, dop, lse, kv_idx, kv_cnt, kcap, scale, dqp, dkp, dvp, ws,

@@ -61,6 +61,9 @@ class DfsLayer:
         else:
             self.scores = None
             self.ws = None
+        # longest rows first for list lengths that vary from row to row
+        self.work_order = (torch.empty(s.B * s.nh * s.nb, dtype=torch.int32, device=dev)
+                           if mode in ("threshold", "global") else None)
         self._index_built = False
         self._bwd = None
         self._pipe = None
@@ -90,19 +93,35 @@ class DfsLayer:
         if self.mode not in STATIC_MODES:
             lib.dfs_block_score(self.shape, self.qp, self.kp, self.scale, self.scores, self.ws, stream)
         lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
+        self._build_order(stream)
+
+    def _build_order(self, stream=None):
+        if self.work_order is not None:
+            lib.dfs_attn_order(self.shape, self.kv_cnt, self.kcap, self.work_order, stream)
 
     def attend(self, stream=None, out=None):
+        """Attention and the inverse reorder into ``out`` (default: the
+        layer's). Without an LSE (inference) the reorder is fused into the
+        attention epilogue; with one, O is kept in curve order in ``op`` for
+        the backward and scattered by a separate kernel."""
+        dst = self.out if out is None else out
+        if self.lse is None and not self.frame_exact:
+            self.attention(stream, out=dst, perm=self.perm)
+            return
         self.attention(stream)
-        lib.dfs_unperm(self.shape, self.perm, self.op, self.out if out is None else out, stream)
+        lib.dfs_unperm(self.shape, self.perm, self.op, dst, stream)
 
-    def attention(self, stream=None):
-        """The attention kernel alone (curve order, into ``op``)."""
+    def attention(self, stream=None, out=None, perm=None):
+        """The attention kernel alone: into ``op`` (curve order), or with
+        ``perm`` straight into the raster tensor ``out``. Rows of uneven list
+        lengths (threshold, global) run in the layer's work order."""
         if self.frame_exact:
             lib.dfs_sparse_attn_lvsa_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt,
                                          self.kcap, self.scale, self.params, self.op, self.lse, stream)
         else:
-            lib.dfs_sparse_attn_fwd(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt, self.kcap,
-                                    self.scale, self.op, self.lse, stream)
+            lib.dfs_sparse_attn_fwd_ex(self.shape, self.qp, self.kp, self.vp, self.kv_idx, self.kv_cnt, self.kcap,
+                                       self.scale, self.op if out is None else out, self.lse, perm=perm,
+                                       order=self.work_order, stream=stream)
 
     def permute_pooled(self, q, k, v, stream=None):
         """Reorder Q, K, V and pool Q, K into the score workspace in one pass."""
@@ -118,6 +137,7 @@ class DfsLayer:
             self.permute_pooled(q, k, v, stream)
             lib.dfs_block_score_pooled(self.shape, self.scale, self.scores, self.ws, stream)
             lib.dfs_select_mask(self.shape, self.scores, self.params, self.kv_idx, self.kv_cnt, self.kcap, stream)
+            self._build_order(stream)
         else:
             self.permute(q, k, v, stream)
             if refresh_mask:

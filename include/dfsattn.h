@@ -226,6 +226,35 @@ int dfs_sparse_attn_fwd(const dfs_shape *shape, const void *qp, const void *kp, 
                         const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
                         void *op, float *lse, dfs_stream_t stream);
 
+/* Options of dfs_sparse_attn_fwd_ex (NULL members: the defaults). */
+typedef struct {
+  /* perm (int32 [N], device; the index of dfs_hilbert_perm): write the row
+   * of curve position i straight to its raster place o[b, perm[i], h, :],
+   * o bf16 [B, N, nh, D] -- the inverse reorder of dfs_unperm fused into
+   * the attention epilogue. NULL: o is op, curve order [B, nh, N, D].    */
+  const int32_t *perm;
+  /* order (int32 [B * nh * nb], device; a permutation of the query rows
+   * (b * nh + h) * nb + I, e.g. from dfs_attn_order): CTA c computes rows
+   * order[2c] and order[2c + 1]. Only the scheduling changes; every row's
+   * result is bitwise the same. NULL: CTA (x, b * nh + h) takes blocks
+   * 2x, 2x + 1 of that head.                                              */
+  const int32_t *order;
+} dfs_attn_opts;
+
+/* dfs_sparse_attn_fwd_ex -- dfs_sparse_attn_fwd with the options above.
+ * lse, if given, stays in curve order.                                     */
+int dfs_sparse_attn_fwd_ex(const dfs_shape *shape, const void *qp, const void *kp, const void *vp,
+                           const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
+                           const dfs_attn_opts *opts, void *o, float *lse, dfs_stream_t stream);
+
+/* dfs_attn_order -- a work order for dfs_attn_opts.order: the query rows
+ * sorted by kept count (kv_cnt clamped to [0, min(kcap, nb)]), largest
+ * first, so the longest rows start first and the two rows of a CTA have
+ * equal work (longest-processing-time first for lists of uneven length,
+ * as threshold and global selection make). Rows of equal count keep their
+ * order within each 32-row chunk. One CTA, no workspace.                   */
+int dfs_attn_order(const dfs_shape *shape, const int32_t *kv_cnt, int kcap, int32_t *order, dfs_stream_t stream);
+
 /* dfs_sparse_attn_lvsa_fwd -- frame-exact LVSA attention (LVSA: Training-Free
  * Sparse Attention for Long Video Diffusion, section 2).
  *

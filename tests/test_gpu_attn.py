@@ -139,3 +139,60 @@ def test_constant_v(lib):
     idx[..., 0] = np.where(idx[..., 0] < 0, 0, idx[..., 0])
     got, _ = _run(lib, q, k, v, idx, cnt, D, blk, N)
     assert np.abs(got - 0.75).max() < 4e-3
+
+
+@pytest.mark.parametrize("grid,D", [((3, 7, 11), 64), ((8, 16, 16), 128), ((21, 30, 52), 128)])
+def test_scatter_epilogue_equals_fwd_then_unperm(lib, grid, D):
+    """The fused inverse reorder writes, bit for bit, what the curve-order
+    forward followed by dfs_unperm writes."""
+    from oracle import hilbert
+    T, H, W = grid
+    N, nh, blk = T * H * W, 2, 128
+    s = lib.Shape(1, nh, D, T, H, W, blk, 16)
+    nb = s.nb
+    rng = np.random.default_rng(N)
+    idx, cnt = _lists(rng, 1, nh, nb, min(nb, 6))
+    g = torch.Generator().manual_seed(N)
+    qp, kp, vp = ((torch.randn((1, nh, N, D), generator=g)).to(torch.bfloat16).cuda() for _ in range(3))
+    perm = torch.from_numpy(hilbert.make_perm("hilbert3d", T, H, W)[0].astype(np.int32)).cuda()
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    op = torch.empty_like(qp)
+    lse_a = torch.empty((1, nh, N), dtype=torch.float32, device="cuda")
+    lse_b = torch.empty_like(lse_a)
+    lib.dfs_sparse_attn_fwd(s, qp, kp, vp, it, ct, idx.shape[-1], 0.0, op, lse_a)
+    ref = torch.empty((1, N, nh, D), dtype=torch.bfloat16, device="cuda")
+    lib.dfs_unperm(s, perm, op, ref)
+    out = torch.full_like(ref, float("nan"))
+    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, idx.shape[-1], 0.0, out, lse_b, perm=perm)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(lse_a, lse_b)
+
+
+@pytest.mark.parametrize("B,nh,D,N,kcap", [(1, 3, 128, 5000, 20), (2, 2, 64, 3000, 24)])
+def test_work_order_changes_nothing(lib, B, nh, D, N, kcap):
+    """Rows run in count order (dfs_attn_order, dfs_attn_opts.order) give
+    bit for bit the rows of the default order; the order is a permutation
+    sorted by kept count, largest first."""
+    blk = 128
+    nb = -(-N // blk)
+    rng = np.random.default_rng(B * N)
+    idx, cnt = _lists(rng, B, nh, nb, kcap)
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, 16)
+    g = torch.Generator().manual_seed(N + D)
+    qp, kp, vp = ((torch.randn((B, nh, N, D), generator=g)).to(torch.bfloat16).cuda() for _ in range(3))
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    order = torch.full((B * nh * nb,), -1, dtype=torch.int32, device="cuda")
+    lib.dfs_attn_order(s, ct, kcap, order)
+    a, b = torch.empty_like(qp), torch.empty_like(qp)
+    la = torch.empty((B, nh, N), dtype=torch.float32, device="cuda")
+    lb = torch.empty_like(la)
+    lib.dfs_sparse_attn_fwd(s, qp, kp, vp, it, ct, kcap, 0.0, a, la)
+    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, b, lb, order=order)
+    torch.cuda.synchronize()
+    o = order.cpu().numpy()
+    assert np.array_equal(np.sort(o), np.arange(B * nh * nb))
+    counts = cnt.reshape(-1)[o]
+    assert (np.diff(counts) <= 0).all()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(la, lb)
