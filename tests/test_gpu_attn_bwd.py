@@ -191,3 +191,42 @@ def test_layer_backward_wan_sampled(lib):
     _check((np.concatenate(got_q), np.concatenate(got_kv)[:, :wl.D], np.concatenate(got_kv)[:, wl.D:]),
            (np.concatenate(ref_q), np.concatenate(ref_kv)[:, :wl.D], np.concatenate(ref_kv)[:, wl.D:]),
            "Wan layer sampled")
+
+
+def test_layer_backward_hunyuan_sampled(lib):
+    """The threshold-selected Hunyuan-shaped layer (24 heads, 118,800
+    tokens, uneven list lengths): dQ on sampled query blocks and dK/dV on
+    sampled key blocks (from every query block that keeps them), one head."""
+    import synth
+    import block_sparse_attention_36_b200 as bsa
+    wl = synth.WORKLOADS["hunyuan_layer"]
+    qkv = synth.workload_inputs(wl)
+    s = bsa.Shape(wl.B, wl.nh, wl.D, wl.T, wl.H, wl.W, wl.blk, wl.sb)
+    layer = bsa.DfsLayer(s, order=wl.order, mode="threshold", cap=wl.ratio_count(wl.cap_num), tau=wl.tau,
+                         want_lse=True)
+    layer.forward(*(qkv[n].cuda() for n in ("q", "k", "v")))
+    g = torch.Generator().manual_seed(22)
+    dout = (torch.randn((wl.B, wl.N, wl.nh, wl.D), generator=g) * 0.5).to(torch.bfloat16)
+    dq, dk, dv = layer.backward(dout.cuda())
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == 0
+    perm = torch.from_numpy(layer.perm.cpu().numpy().astype(np.int64))
+    h = 7
+    ii, cc = layer.kv_idx.cpu().numpy()[:, h:h + 1], layer.kv_cnt.cpu().numpy()[:, h:h + 1]
+    cur = [x[0, perm, h, :].double().numpy()[None, None] for x in (qkv["q"], qkv["k"], qkv["v"], dout)]
+    gq, gk, gv = (x.cpu()[0, perm, h, :].float().numpy() for x in (dq, dk, dv))
+    rng = np.random.default_rng(5)
+    Is = [0, wl.nb - 1] + [int(x) for x in rng.integers(0, wl.nb, 2)]
+    rq, _, _ = attention.block_sparse_attention_bwd(*cur, ii, cc, wl.blk, rows=[(0, 0, I) for I in Is])
+    Js = [wl.nb - 1, int(rng.integers(0, wl.nb))]
+    keep = [set(ii[0, 0, I, :cc[0, 0, I]].tolist()) for I in range(wl.nb)]
+    got_q = np.concatenate([gq[I * wl.blk:min(wl.N, I * wl.blk + wl.blk)] for I in Is])
+    ref_q = np.concatenate([rq[0, 0, I * wl.blk:min(wl.N, I * wl.blk + wl.blk)] for I in Is])
+    got_k, got_v, ref_k, ref_v = [], [], [], []
+    for J in Js:
+        rows = [(0, 0, I) for I in range(wl.nb) if J in keep[I]]
+        _, rk, rv = attention.block_sparse_attention_bwd(*cur, ii, cc, wl.blk, rows=rows)
+        lo, hi = J * wl.blk, min(wl.N, J * wl.blk + wl.blk)
+        got_k.append(gk[lo:hi]); got_v.append(gv[lo:hi]); ref_k.append(rk[0, 0, lo:hi]); ref_v.append(rv[0, 0, lo:hi])
+    _check((got_q, np.concatenate(got_k), np.concatenate(got_v)),
+           (ref_q, np.concatenate(ref_k), np.concatenate(ref_v)), "Hunyuan layer sampled")
