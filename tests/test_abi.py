@@ -88,3 +88,43 @@ def test_argument_errors_need_no_gpu(lib):
     assert L.dfs_sparse_attn_fwd(ctypes.byref(sh), fake, fake, odd, fake, fake, 4, 0.0, fake, None, None) == -3
     zero = _shape_c(lib, T=0)
     assert L.dfs_unperm(ctypes.byref(zero), fake, fake, fake, None) == -1
+
+
+def test_argument_errors_of_later_entry_points(lib):
+    """Extended forward, work order, frame-exact LVSA, backward, no-alloc
+    scoring and the workspace query: host-side checks only."""
+    L = lib.LIB
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    odd = P((1 << 20) + 2)
+    sh = _shape_c(lib)                     # blk 64
+    sh128 = _shape_c(lib, blk=128)
+    opts = lib._AttnOpts(None, None)
+    assert L.dfs_sparse_attn_fwd_ex(ctypes.byref(sh), fake, fake, fake, fake, fake, 0, 0.0, ctypes.byref(opts),
+                                    fake, None, None) == -1
+    assert L.dfs_sparse_attn_fwd_ex(ctypes.byref(sh), fake, fake, fake, fake, fake, 4, 0.0, ctypes.byref(opts),
+                                    odd, None, None) == -3
+    assert L.dfs_attn_order(ctypes.byref(sh), None, 4, fake, None) == -1
+    assert L.dfs_attn_order(ctypes.byref(sh), fake, 0, fake, None) == -1
+    prm = lib.select_params("lvsa", lvsa_T_per=0, lvsa_C=4)
+    assert L.dfs_sparse_attn_lvsa_fwd(ctypes.byref(sh), fake, fake, fake, fake, fake, 4, 0.0, ctypes.byref(prm),
+                                      fake, None, None) == -1
+    prm = lib.select_params("lvsa", lvsa_T_per=2, lvsa_C=4)
+    small_frames = _shape_c(lib, H=4, W=8)             # H * W = 32 < blk = 64
+    assert L.dfs_sparse_attn_lvsa_fwd(ctypes.byref(small_frames), fake, fake, fake, fake, fake, 4, 0.0,
+                                      ctypes.byref(prm), fake, None, None) == -2
+    need = lib.dfs_workspace_bytes(lib.Shape(1, 2, 64, 8, 16, 16, 128, 16), lib.DFS_WS_ATTN_BWD)
+    assert need > 0
+    args = [fake] * 8
+    assert L.dfs_sparse_attn_bwd(ctypes.byref(sh), *args, 4, 0.0, fake, fake, fake, fake, 1 << 30, None) == -2
+    assert L.dfs_sparse_attn_bwd(ctypes.byref(sh128), *args, 4, 0.0, fake, fake, fake, fake, need - 1, None) == -6
+    assert L.dfs_sparse_attn_bwd(ctypes.byref(sh128), *args[:5], None, *args[6:], 4, 0.0, fake, fake, fake, fake,
+                                 need, None) == -1
+    assert L.dfs_sparse_attn_bwd(ctypes.byref(sh128), *args, 4, 0.0, fake, fake, fake, P((1 << 20) + 16), need,
+                                 None) == -3
+    prm = lib.select_params("radial", radial_w0=-1)
+    assert L.dfs_select_mask(ctypes.byref(sh), None, ctypes.byref(prm), fake, fake, 8, None) == -1
+    prm = lib.select_params("radial", radial_w0=8, radial_lambda=-0.5)
+    assert L.dfs_select_mask(ctypes.byref(sh), None, ctypes.byref(prm), fake, fake, 8, None) == -1
+    big = _shape_c(lib, B=8, nh=16, T=64, H=64, W=64, blk=128, sb=32)   # pooled means >> 32 MiB
+    assert L.dfs_block_score_noalloc(ctypes.byref(big), fake, fake, 0.0, fake, None) == -6
