@@ -54,6 +54,28 @@ ATTN_TRAFFIC = {"wan_1p3b_layer": (298_673_152 + 82_699_520, "99ab3bb278d64954")
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 
+# dram read + write of one backward call (all its launches) on the Wan layer,
+# from a one-pass ncu capture of these sources
+BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_541_248 + 263_128_064, "9251d62b2020bb22")}
+BWD_SOURCES = ("attn_bwd.cu", "sm100_ptx.cuh", "common.cuh", "tmap.cuh")
+
+
+def sources_hash(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "block_sparse_attention_36_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def bwd_traffic(workload):
+    entry = BWD_TRAFFIC.get(workload)
+    if entry is None or entry[1] != sources_hash(BWD_SOURCES):
+        return None
+    return entry[0]
+
+
 def attn_sources_hash():
     import hashlib
     h = hashlib.sha256()
@@ -443,7 +465,8 @@ def run_backward(args):
                        "parallelism": f"replicas x{world} (independent layer per GPU)"},
             "roofline": {"kernel": "dfs_sparse_attn_bwd (prep, mask bits, transpose, dQ pass, dK/dV pass)",
                          "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4), "peak_source": f"{src} bf16 burst", "traffic": None},
+                         "frac": round(achieved / peak, 4), "peak_source": f"{src} bf16 burst",
+                         "traffic": bwd_traffic(wl.name)},
             "e2e": {"value": round(sum_over_ranks(flops_step, world) / (e2e_ms * 1e-3) / 1e12, 3),
                     "unit": "TFLOP/s (kept-block backward, whole step)", "ms_per_step": round(e2e_ms, 3),
                     "h2d_bytes_per_step": int(dh.numel() * dh.element_size()),
