@@ -89,6 +89,15 @@ constexpr int kPad = 4;      // smem row padding (floats)
 // memory into registers while the current one is multiplied, and the 8 x 8
 // register tile is updated with paired fp32 FMAs (two columns per
 // instruction; each sum is still one fp32 fma chain over d, as before).
+// For R <= 4 a thread's eight columns are two runs of four, 4tx and
+// 64 + 4tx, so that a warp's 16-byte column loads are contiguous (without
+// bank conflicts); an R x R pool group then stays inside one run. For
+// R = 8 the eight columns are consecutive.
+template <int R>
+__device__ __forceinline__ int score_col(int tx, int jj) {
+  return R <= 4 ? (jj < 4 ? tx * 4 + jj : 64 + tx * 4 + jj - 4) : tx * 8 + jj;
+}
+
 template <int R>
 __global__ void __launch_bounds__(256, 2)
 score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
@@ -141,8 +150,8 @@ score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
     for (int kk = 0; kk < kKStep; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8]);
       const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][score_col<R>(tx, 0)]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][score_col<R>(tx, 4)]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float2 b[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
                            make_float2(b1.z, b1.w)};
@@ -171,12 +180,12 @@ score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
       for (int i = 0; i < R; ++i)
 #pragma unroll
         for (int j = 0; j < R; ++j) {
-          const int sr = row0 + ty * 8 + gi * R + i, sc = col0 + tx * 8 + gj * R + j;
+          const int sr = row0 + ty * 8 + gi * R + i, sc = col0 + score_col<R>(tx, gj * R + j);
           const int cc = gj * R + j;
           const float2 pr = acc[gi * R + i][cc >> 1];
           if (sr < nsb && sc < nsb) m = fmaxf(m, (cc & 1) ? pr.y : pr.x);
         }
-      const int I = (row0 + ty * 8) / R + gi, J = (col0 + tx * 8) / R + gj;
+      const int I = (row0 + ty * 8) / R + gi, J = (col0 + score_col<R>(tx, gj * R)) / R;
       if (I < nb && J < nb) scores[(bh * nb + I) * (long long)nb + J] = m * scale;
     }
   }
