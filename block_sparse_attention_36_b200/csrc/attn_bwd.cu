@@ -672,11 +672,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       for (int c = 0; c < 2; ++c) {
         uint32_t sr[32], po[16];
         tmem_ld32(s_addr + 32 * c, sr);
+        // this chunk's 32 constants, loaded while the tensor-memory load is in flight
+        float4 nl4[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) nl4[v] = *reinterpret_cast<const float4*>(nl + 64 * g + 32 * c + 4 * v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int q = 64 * g + 32 * c + 2 * e;
-          const float2 nl2 = *reinterpret_cast<const float2*>(nl + q);
+          const float2 nl2 = (e & 1) ? make_float2(nl4[e >> 1].z, nl4[e >> 1].w) : make_float2(nl4[e >> 1].x, nl4[e >> 1].y);
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sc2, nl2);
           pv[32 * c + 2 * e] = ex2(x.x);
           pv[32 * c + 2 * e + 1] = ex2(x.y);
@@ -698,11 +701,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       for (int c = 0; c < 2; ++c) {
         uint32_t pr[32], so[16];
         tmem_ld32(p_addr + 32 * c, pr);
+        float4 nd4[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) nd4[v] = *reinterpret_cast<const float4*>(nd + 64 * g + 32 * c + 4 * v);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int q = 64 * g + 32 * c + 2 * e;
-          const float2 nd2 = *reinterpret_cast<const float2*>(nd + q);
+          const float2 nd2 = (e & 1) ? make_float2(nd4[e >> 1].z, nd4[e >> 1].w) : make_float2(nd4[e >> 1].x, nd4[e >> 1].y);
           const float2 t = __fadd2_rn(make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])), nd2);
           const float2 ds = __fmul2_rn(make_float2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]), t);
           so[e] = pack_bf16x2(ds.x, ds.y);
