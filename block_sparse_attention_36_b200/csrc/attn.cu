@@ -73,7 +73,7 @@ struct Cfg {
 struct __align__(8) Barriers {
   uint64_t q_full[2];
   uint64_t kv_full[kRing], kv_empty[kRing];
-  uint64_t s_full[2], p_full[2], o_final[2];
+  uint64_t s_full[2], p_half[2], p_full[2], o_final[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -95,11 +95,13 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t d
 
 // O (+)= P V for one query tile: P (bf16) from tensor memory, V MN-major in
 // shared memory; BLK/16 MMAs of K = 16.
-template <int D, int BLK>
+// K steps [KK0, KK1) only: the first half of P can be consumed while the
+// second half is still being formed.
+template <int D, int BLK, int KK0, int KK1>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(kQRows, D, 1);
 #pragma unroll
-  for (int kk = 0; kk < BLK / 16; ++kk)
+  for (int kk = KK0; kk < KK1; ++kk)
     mma_ts_warp(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -160,6 +162,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->q_full[x], 1);
       mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_half[x], 4);
       mbar_init(&bars->p_full[x], 4);
       mbar_init(&bars->o_final[x], 1);
     }
@@ -309,12 +312,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // P_X was written by other threads with tcgen05.st: order this
             // thread's MMAs after their arrival. (TMA-filled tiles need no
             // fence: the mbarrier transaction count orders them.)
-            if (!mbar_wait_bounded(&bars->p_full[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-            tc_fence_after();
             const int st = t % kRing;
-            if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-            issue_pv<D, BLK>(tmem + C::o_col(x), tmem + C::s_col(x), dv + (uint64_t)((st * C::kTileBytes) >> 4),
-                             step > 0);
+            const uint64_t dvs = dv + (uint64_t)((st * C::kTileBytes) >> 4);
+            if (BLK == 128) {
+              // keys 0-63 of P(step) first, while the softmax forms keys 64-127
+              if (!mbar_wait_bounded(&bars->p_half[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              tc_fence_after();
+              if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              issue_pv<D, BLK, 0, BLK / 32>(tmem + C::o_col(x), tmem + C::s_col(x), dvs, step > 0);
+              if (!mbar_wait_bounded(&bars->p_full[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv<D, BLK, BLK / 32, BLK / 16>(tmem + C::o_col(x), tmem + C::s_col(x), dvs, true);
+            } else {
+              if (!mbar_wait_bounded(&bars->p_full[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              tc_fence_after();
+              if (!mbar_wait_bounded(&bars->kv_full[st], (uint32_t)((t / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              issue_pv<D, BLK, 0, BLK / 16>(tmem + C::o_col(x), tmem + C::s_col(x), dvs, step > 0);
+            }
             mma_commit_warp(&bars->kv_empty[st]);
             ++t;
           }
@@ -432,12 +446,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           packed[e] = pack_bf16x2(p2.x, p2.y);
         }
         tmem_st32(s_addr + c * 32, packed);
+        if (BLK == 128 && c == 0 && !rescale) {
+          // keys 0-63 of P are in place: release them to the MMAs while the
+          // rest is formed (a warp that rescales O releases them after that)
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->p_half[x]);
+        }
       }
       const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
       const float2 a = __fadd2_rn(a01, a23);
       const float rs = a.x + a.y;
       // O_X may be rescaled here: s_full(j) was committed after PV_X(j-1)
-      // by the same thread, so PV_X(j-1) has completed.
+      // by the same thread, so PV_X(j-1) has completed, and no MMA of PV_X(j)
+      // starts before this warp's arrival on p_half.
       if (rescale) {
         // (a row with no unmasked key yet has O = 0 and l = 0)
         const float alpha = (FRAME && m == -INFINITY) ? 0.f : ex2(m - m_use);
@@ -456,6 +479,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_st32(o_addr + c * 32, raw);
         }
         l *= alpha;
+        if (BLK == 128) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->p_half[x]);
+        }
       }
       tmem_wait_st();
       m = m_use;
