@@ -50,13 +50,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch from one ncu capture
 # (profiles/attn_fwd_<workload>.md), valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
-ATTN_TRAFFIC = {"wan_1p3b_layer": (298_673_152 + 82_699_520, "99ab3bb278d64954")}
+ATTN_TRAFFIC = {"wan_1p3b_layer": (298_970_368 + 82_699_008, "c33ffab6d4104243")}
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 
 # dram read + write of one backward call (all its launches) on the Wan layer,
 # from a one-pass ncu capture of these sources
-BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_541_248 + 263_128_064, "9251d62b2020bb22")}
+BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_195_136 + 263_207_424, "52bad2f1fdf8b4eb")}
 BWD_SOURCES = ("attn_bwd.cu", "sm100_ptx.cuh", "common.cuh", "tmap.cuh")
 
 
