@@ -173,6 +173,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
+    // Q of each existing slot depends only on its block index: start both
+    // loads now, while the lists are being staged.
+    for (int x = 0; x < 2; ++x) {
+      if (slot_I(x) >= nb) continue;
+      mbar_arrive_expect_tx(&bars->q_full[x], C::kQBytes);
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_3d(smem + C::kQOff + x * C::kQBytes + c * (kQRows * 128), &tm_q, &bars->q_full[x], c * 64,
+                    slot_I(x) * BLK, slot_bh(x));
+    }
   }
   if (warp == 2 || warp == 3) {
     // Compact the slot's kept list into shared memory, dropping invalid indices.
@@ -182,14 +191,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool bad = false;
     if (I < nb) {
       const long long row_id = (long long)slot_bh(x) * nb + I;
-      int cnt = kv_cnt[row_id];
-      cnt = max(0, min(cnt, min(kcap, max_list)));
       const int32_t* src = kv_idx + row_id * (long long)kcap;
+      const int lim = min(kcap, max_list);
+      const int J_first = lane < lim ? src[lane] : -1;    // fetched alongside the count
+      int cnt = kv_cnt[row_id];
+      cnt = max(0, min(cnt, lim));
       int32_t* dst = lists + x * max_list;
       for (int j0 = 0; j0 < cnt; j0 += 32) {
         const int j = j0 + lane;
         int J = -1;
-        if (j < cnt) J = src[j];
+        if (j < cnt) J = (j0 == 0) ? J_first : src[j];
         const bool ok = (j < cnt) && J >= 0 && J < nb;
         bad |= (j < cnt) && !ok;
         const unsigned m = __ballot_sync(0xffffffffu, ok);
@@ -243,13 +254,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         prefetch_tensor_map(&tm_k);
         prefetch_tensor_map(&tm_v);
       }
-      for (int x = 0; x < 2; ++x) {
-        if (n[x] == 0) continue;
-        mbar_arrive_expect_tx_warp(&bars->q_full[x], C::kQBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d_warp(smem + C::kQOff + x * C::kQBytes + c * (kQRows * 128), &tm_q, &bars->q_full[x], c * 64,
-                           slot_I(x) * BLK, slot_bh(x));
-      }
       // Same step order as the MMA issuer: step -1 loads K_A(0), K_B(0); step
       // j loads, per slot, V(j) and then K(j+1).
       int t = 0;  // ring tiles loaded so far
@@ -285,7 +289,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int u = max(0, t - kRing); u < t; ++u)
         mbar_wait_timed(&bars->kv_full[u % kRing], (uint32_t)((u / kRing) & 1), kDrainLimit);
       for (int x = 0; x < 2; ++x)
-        if (n[x] > 0) mbar_wait_timed(&bars->q_full[x], 0, kDrainLimit);
+        if (slot_I(x) < nb) mbar_wait_timed(&bars->q_full[x], 0, kDrainLimit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
