@@ -6,13 +6,16 @@
 // contiguous token blocks.
 //
 // A CTA owns two query tiles ("slots" A and B: query blocks 2x and 2x+1 of
-// one head), each with its own kept list. While the softmax of one slot
-// runs, the tensor pipe works on the other slot's products, so neither the
-// tensor pipe nor the exponential units wait on each other for long.
+// one head, or rows order[2x], order[2x+1] of a work order), each with its
+// own kept list. While the softmax of one slot runs, the tensor pipe works
+// on the other slot's products, so neither the tensor pipe nor the
+// exponential units wait on each other for long.
 // Warp roles (384 threads, three warpgroups):
-//   warp 0     TMA producer: Q_A, Q_B, then the K and V tiles of both lists
-//              into a 4-stage ring, in exactly the order the MMAs consume
-//              them (128-byte swizzled tiles, no multicast).
+//   thread 0   initialises the barriers and starts the Q_A, Q_B loads at
+//              once (they depend only on the block index).
+//   warp 0     TMA producer: the K and V tiles of both lists into a 4-stage
+//              ring, in exactly the order the MMAs consume them (128-byte
+//              swizzled tiles, no multicast).
 //   warp 1     owns tensor memory; one lane issues the tcgen05 MMAs, per
 //              slot X and kept block j:
 //                S_X = Q_X K_j^T  (SS)            into TMEM S_X
@@ -20,6 +23,9 @@
 //              ordered S_A(0) S_B(0), then per j: PV_A(j) S_A(j+1)
 //              PV_B(j) S_B(j+1); S_X(j+1) overwrites P_X(j) only after
 //              PV_X(j) read it (tcgen05 MMAs of one thread run in order).
+//              With 128-key blocks, PV_X(j) starts on keys 0-63 of P as
+//              soon as the softmax releases them (p_half) and finishes on
+//              keys 64-127 after p_full.
 //   warps 2-3  compact the two kept lists into shared memory, then idle.
 //   warps 4-7  softmax of slot A, warps 8-11 softmax of slot B: one thread
 //              per query row; fp32 online softmax on S read from TMEM,
@@ -27,7 +33,8 @@
 //              only when a warp's running maximum grows by more than 2^8
 //              (an older maximum stays exact as long as P and the row sum
 //              use the same one); epilogue normalises O_X and stores bf16
-//              rows and the log-sum-exp.
+//              rows (in curve order, or straight to raster order through
+//              perm) and the log-sum-exp.
 // Tensor memory: S_A | S_B | O_A | O_B (BLK, BLK, D, D fp32 columns).
 // Every mbarrier wait is bounded (DFS_FLAG_WAIT_TIMEOUT, early return);
 // copies and MMAs in flight are drained before tensor memory is released.
