@@ -9,11 +9,16 @@
 //
 // Kernel 1 (pool): one warp per sub-block streams its sb x D bf16 tile with
 // 16-byte loads (8 values per lane) and keeps fp32 sums; HBM-bound.
-// Kernel 2 (score): a 128 x 128 tile of pooled logits per CTA computed with
-// fp32 FMAs from shared-memory staged operands (8 x 8 per thread), followed
-// by the r x r max-pool inside each thread's registers (r = blk/sb divides
-// 8, so every pooled group lies inside one thread's 8 x 8 patch).
+// Kernel 2 (score): the pooled logits of a 128 x 256 tile of (query,
+// key) sub-blocks are one dense product qbar_tile . kbar_tile^T over D, run
+// on the tensor cores (tcgen05, kind::tf32, accumulator in tensor memory).
+// Each fp32 operand x is split into x_hi = tf32(x) and x_lo = tf32(x - x_hi)
+// and the product is taken as a_lo b_hi + a_hi b_lo + a_hi b_hi (the
+// dropped a_lo b_lo and the rounding of the lo parts are below 2^-22 of
+// |a||b| per term, i.e. fp32-level accuracy). The r x r max-pool runs in the
+// epilogue: r columns inside a thread's row, r rows across r lanes.
 #include "common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace {
 
@@ -80,115 +85,192 @@ pool_kernel(const __nv_bfloat16* __restrict__ qp, const __nv_bfloat16* __restric
   }
 }
 
-constexpr int kTile = 128;   // sub-blocks per tile side
-constexpr int kKStep = 16;   // head-dim slice staged per iteration
-constexpr int kPad = 4;      // smem row padding (floats)
+using namespace dfs::sm100;
+
+constexpr int kSM = 128;                    // query sub-blocks per tile (MMA M)
+constexpr int kSN = 256;                    // key sub-blocks per tile (MMA N)
+constexpr int kScoreThreads = 256;
+constexpr int kQSlab = kSM * 128;           // one 32-column fp32 slab of the query tile, bytes
+constexpr int kKSlab = kSN * 128;           // the same for the key tile
+constexpr int kScoreSmem = 1024 + 2 * kQSlab + 2 * kKSlab;   // + alignment slack
+constexpr long long kScoreWait = 2000000000ll;   // SM clock cycles per wait (about 1 s)
 
 // scores[bh, I, J] = scale * max_{i in I, j in J} sum_d qbar[bh,i,d] kbar[bh,j,d]
-// Two shared-memory buffers: the next head-dim slice is read from global
-// memory into registers while the current one is multiplied, and the 8 x 8
-// register tile is updated with paired fp32 FMAs (two columns per
-// instruction; each sum is still one fp32 fma chain over d, as before).
-// For R <= 4 a thread's eight columns are two runs of four, 4tx and
-// 64 + 4tx, so that a warp's 16-byte column loads are contiguous (without
-// bank conflicts); an R x R pool group then stays inside one run. For
-// R = 8 the eight columns are consecutive.
-template <int R>
-__device__ __forceinline__ int score_col(int tx, int jj) {
-  return R <= 4 ? (jj < 4 ? tx * 4 + jj : 64 + tx * 4 + jj - 4) : tx * 8 + jj;
-}
-
-template <int R>
-__global__ void __launch_bounds__(256, 2)
-score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-             float* __restrict__ scores, int D, int nsb, int nb, float scale) {
-  __shared__ __align__(16) float As[2][kKStep][kTile + kPad];
-  __shared__ __align__(16) float Bs[2][kKStep][kTile + kPad];
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+// One CTA per 128 x 256 tile of sub-block pairs (two CTAs per SM, 256
+// tensor-memory columns each). The head dimension is walked in slabs of 32
+// fp32 columns (one 128-byte row per sub-block): every thread loads its
+// share of the slab from global memory into registers, splits it into tf32
+// hi and lo parts and stores both into 128-byte-swizzled shared-memory
+// tiles (the 16-byte chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4),
+// the layout the MMA descriptors expect); one warp then issues the slab's
+// 3 x 4 MMAs (K = 8 each) and commits them, and the next slab's loads are
+// in flight while they run.
+template <int D, int R>
+__global__ void __launch_bounds__(kScoreThreads, 2)
+score_tc_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, float* __restrict__ scores,
+                int nsb, int nb, float scale) {
+  extern __shared__ uint8_t score_smem[];
+  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  constexpr int kSlabs = D / 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long bh = blockIdx.z;
-  const int row0 = blockIdx.y * kTile, col0 = blockIdx.x * kTile;
+  const int row0 = blockIdx.y * kSM, col0 = blockIdx.x * kSN;
+  const uint32_t raw = smem_addr(score_smem);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* tiles = score_smem + (base - raw);
+  uint8_t* q_hi = tiles;
+  uint8_t* q_lo = tiles + kQSlab;
+  uint8_t* k_hi = tiles + 2 * kQSlab;
+  uint8_t* k_lo = k_hi + kKSlab;
+
+  if (warp == 0) tmem_alloc(&tmem_slot, 256);
+  if (tid == 0) {
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+
   const float* qa = qbar + bh * (long long)nsb * D;
   const float* ka = kbar + bh * (long long)nsb * D;
-  float2 acc[8][4];
+  // slab s: query rows r < 128 and key rows r < 256, eight 16-byte chunks
+  // per row; thread t takes the chunks t, t + 256, ... of the slab
+  float4 rq[kSM * 8 / kScoreThreads], rk[kSN * 8 / kScoreThreads];
+  auto fetch = [&](int slab) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+    for (int u = 0; u < kSM * 8 / kScoreThreads; ++u) {
+      const int f = tid + u * kScoreThreads, r = f >> 3, c = f & 7;
+      rq[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (row0 + r < nsb) rq[u] = __ldg(reinterpret_cast<const float4*>(qa + (long long)(row0 + r) * D + slab * 32 + c * 4));
+    }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
+    for (int u = 0; u < kSN * 8 / kScoreThreads; ++u) {
+      const int f = tid + u * kScoreThreads, r = f >> 3, c = f & 7;
+      rk[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (col0 + r < nsb) rk[u] = __ldg(reinterpret_cast<const float4*>(ka + (long long)(col0 + r) * D + slab * 32 + c * 4));
+    }
+  };
+  auto split_store = [&](const float4& x, uint8_t* hi, uint8_t* lo, int f) {
+    const int r = f >> 3, c = f & 7;
+    const int off = r * 128 + ((c ^ (r & 7)) << 4);
+    float4 h, l;
+    h.x = round_tf32(x.x); l.x = round_tf32(x.x - h.x);
+    h.y = round_tf32(x.y); l.y = round_tf32(x.y - h.y);
+    h.z = round_tf32(x.z); l.z = round_tf32(x.z - h.z);
+    h.w = round_tf32(x.w); l.w = round_tf32(x.w - h.w);
+    *reinterpret_cast<float4*>(hi + off) = h;
+    *reinterpret_cast<float4*>(lo + off) = l;
+  };
 
-  float4 ga[2], gb[2];
-  auto fetch = [&](int k0) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int f = tid + u * 256;
-      const int r = f >> 2, c4 = (f & 3) * 4;
-      ga[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      gb[u] = ga[u];
-      if (row0 + r < nsb) ga[u] = *reinterpret_cast<const float4*>(qa + (long long)(row0 + r) * D + k0 + c4);
-      if (col0 + r < nsb) gb[u] = *reinterpret_cast<const float4*>(ka + (long long)(col0 + r) * D + k0 + c4);
-    }
-  };
-  auto stash = [&](int buf) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int f = tid + u * 256;
-      const int r = f >> 2, c4 = (f & 3) * 4;
-      As[buf][c4 + 0][r] = ga[u].x; As[buf][c4 + 1][r] = ga[u].y;
-      As[buf][c4 + 2][r] = ga[u].z; As[buf][c4 + 3][r] = ga[u].w;
-      Bs[buf][c4 + 0][r] = gb[u].x; Bs[buf][c4 + 1][r] = gb[u].y;
-      Bs[buf][c4 + 2][r] = gb[u].z; Bs[buf][c4 + 3][r] = gb[u].w;
-    }
-  };
   fetch(0);
-  stash(0);
+  tc_fence_before();
   __syncthreads();
-  int buf = 0;
-  for (int k0 = 0; k0 < D; k0 += kKStep) {
-    const bool more = k0 + kKStep < D;
-    if (more) fetch(k0 + kKStep);
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  constexpr uint32_t idesc = idesc_tf32_f32(kSM, kSN);
+#pragma unroll 1
+  for (int slab = 0; slab < kSlabs; ++slab) {
+    if (slab > 0) {
+      // the previous slab's MMAs have read the tiles
+      mbar_wait_bounded(&mma_done, (slab - 1) & 1, &abort_flag, kScoreWait);
+      tc_fence_after();
+    }
 #pragma unroll
-    for (int kk = 0; kk < kKStep; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][score_col<R>(tx, 0)]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][score_col<R>(tx, 4)]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float2 b[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
-                           make_float2(b1.z, b1.w)};
+    for (int u = 0; u < kSM * 8 / kScoreThreads; ++u) split_store(rq[u], q_hi, q_lo, tid + u * kScoreThreads);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float2 ai = make_float2(a[i], a[i]);
+    for (int u = 0; u < kSN * 8 / kScoreThreads; ++u) split_store(rk[u], k_hi, k_lo, tid + u * kScoreThreads);
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(ai, b[j], acc[i][j]);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t o = kk * 32;   // K = 8 fp32 columns = 32 bytes along the swizzled row
+        const uint64_t aq_hi = desc_sw128(smem_addr(q_hi) + o, 16, 1024);
+        const uint64_t aq_lo = desc_sw128(smem_addr(q_lo) + o, 16, 1024);
+        const uint64_t bk_hi = desc_sw128(smem_addr(k_hi) + o, 16, 1024);
+        const uint64_t bk_lo = desc_sw128(smem_addr(k_lo) + o, 16, 1024);
+        mma_ss_tf32_warp(tmem, aq_lo, bk_hi, idesc, (slab > 0 || kk > 0) ? 1u : 0u);
+        mma_ss_tf32_warp(tmem, aq_hi, bk_lo, idesc, 1u);
+        mma_ss_tf32_warp(tmem, aq_hi, bk_hi, idesc, 1u);
+      }
+      mma_commit_warp(&mma_done);
+    }
+    if (slab + 1 < kSlabs) fetch(slab + 1);
+  }
+  if (!mbar_wait_bounded(&mma_done, (kSlabs - 1) & 1, &abort_flag, kScoreWait))
+    atomicOr(&g_score_flags, DFS_FLAG_WAIT_TIMEOUT);
+  tc_fence_after();
+
+  // epilogue: warp w reads tensor-memory lanes 32 (w & 3) .. + 31 (its
+  // query sub-block rows) and columns 128 (w >> 2) .. + 127 in chunks of 32
+  const int quarter = warp & 3, half = warp >> 2;
+  const int srow = row0 + quarter * 32 + lane;
+  const bool row_ok = srow < nsb;
+#pragma unroll 1
+  for (int ch = 0; ch < 4; ++ch) {
+    const int cbase = half * 128 + ch * 32;
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)cbase, v);
+    tmem_wait_ld();
+    float m[32 / R];
+#pragma unroll
+    for (int g = 0; g < 32 / R; ++g) {
+      m[g] = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        if (row_ok && col0 + cbase + g * R + j < nsb) m[g] = fmaxf(m[g], __uint_as_float(v[g * R + j]));
+    }
+#pragma unroll
+    for (int off = 1; off < R; off <<= 1)
+#pragma unroll
+      for (int g = 0; g < 32 / R; ++g) m[g] = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], off));
+    const int I = srow / R;
+    if (lane % R == 0 && I < nb) {
+      float* dst = scores + (bh * nb + I) * (long long)nb;
+#pragma unroll
+      for (int g = 0; g < 32 / R; ++g) {
+        const int J = (col0 + cbase) / R + g;
+        if (J < nb) dst[J] = m[g] * scale;
       }
     }
-    if (more) {
-      stash(buf ^ 1);
-      __syncthreads();
-      buf ^= 1;
-    }
   }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    if (abort_flag) mbar_wait_timed(&mma_done, (kSlabs - 1) & 1, kScoreWait);
+    tmem_dealloc(tmem, 256);
+  }
+}
 
-  // r x r max-pool within the 8 x 8 patch; sub-blocks past nsb do not exist.
-  constexpr int G = 8 / R;
-#pragma unroll
-  for (int gi = 0; gi < G; ++gi) {
-#pragma unroll
-    for (int gj = 0; gj < G; ++gj) {
-      float m = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < R; ++i)
-#pragma unroll
-        for (int j = 0; j < R; ++j) {
-          const int sr = row0 + ty * 8 + gi * R + i, sc = col0 + score_col<R>(tx, gj * R + j);
-          const int cc = gj * R + j;
-          const float2 pr = acc[gi * R + i][cc >> 1];
-          if (sr < nsb && sc < nsb) m = fmaxf(m, (cc & 1) ? pr.y : pr.x);
-        }
-      const int I = (row0 + ty * 8) / R + gi, J = (col0 + score_col<R>(tx, gj * R)) / R;
-      if (I < nb && J < nb) scores[(bh * nb + I) * (long long)nb + J] = m * scale;
-    }
+template <int D, int R>
+int launch_score_tc(const dfs::Dims& d, const float* qbar, const float* kbar, float* scores, float scale,
+                    cudaStream_t cs) {
+  if (cudaFuncSetAttribute(score_tc_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem) !=
+      cudaSuccess)
+    return DFS_ERR_CUDA;
+  const dim3 grid((unsigned)((d.nsb + kSN - 1) / kSN), (unsigned)((d.nsb + kSM - 1) / kSM), (unsigned)d.BH);
+  score_tc_kernel<D, R><<<grid, kScoreThreads, kScoreSmem, cs>>>(qbar, kbar, scores, d.nsb, d.nb, scale);
+  return dfs::launch_status();
+}
+
+template <int D>
+int launch_score_d(const dfs::Dims& d, const float* qbar, const float* kbar, float* scores, float scale,
+                   cudaStream_t cs) {
+  switch (d.r) {
+    case 1: return launch_score_tc<D, 1>(d, qbar, kbar, scores, scale, cs);
+    case 2: return launch_score_tc<D, 2>(d, qbar, kbar, scores, scale, cs);
+    case 4: return launch_score_tc<D, 4>(d, qbar, kbar, scores, scale, cs);
+    default: return launch_score_tc<D, 8>(d, qbar, kbar, scores, scale, cs);
   }
+}
+
+// Block scores from pooled means qbar, kbar ([BH, nsb, D] fp32 each).
+int launch_score(const dfs::Dims& d, const float* qbar, const float* kbar, float* scores, float scale,
+                 cudaStream_t cs) {
+  return d.D == 128 ? launch_score_d<128>(d, qbar, kbar, scores, scale, cs)
+                    : launch_score_d<64>(d, qbar, kbar, scores, scale, cs);
 }
 
 }  // namespace
@@ -229,15 +311,7 @@ extern "C" int dfs_block_score(const dfs_shape* shape, const void* qp, const voi
   if (st != DFS_OK) return st;
   const float* qbar = pooled;
   const float* kbar = pooled + d.BH * d.nsb * d.D;
-  const unsigned tiles = (unsigned)((d.nsb + kTile - 1) / kTile);
-  dim3 sg(tiles, tiles, (unsigned)d.BH);
-  switch (d.r) {
-    case 1: score_kernel<1><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    case 2: score_kernel<2><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    case 4: score_kernel<4><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    default: score_kernel<8><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-  }
-  return dfs::launch_status();
+  return launch_score(d, qbar, kbar, scores, scale, cs);
 }
 
 extern "C" int dfs_block_score_pooled(const dfs_shape* shape, float scale, float* scores, const void* ws,
@@ -255,15 +329,7 @@ extern "C" int dfs_block_score_pooled(const dfs_shape* shape, float scale, float
   cudaStream_t cs = (cudaStream_t)stream;
   const float* qbar = (const float*)ws;
   const float* kbar = qbar + d.BH * d.nsb * d.D;
-  const unsigned tiles = (unsigned)((d.nsb + kTile - 1) / kTile);
-  dim3 sg(tiles, tiles, (unsigned)d.BH);
-  switch (d.r) {
-    case 1: score_kernel<1><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    case 2: score_kernel<2><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    case 4: score_kernel<4><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    default: score_kernel<8><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-  }
-  return dfs::launch_status();
+  return launch_score(d, qbar, kbar, scores, scale, cs);
 }
 
 // ---------------------------------------------------------------------------
@@ -330,13 +396,5 @@ extern "C" int dfs_block_score_noalloc(const dfs_shape* shape, const void* qp, c
   if (st != DFS_OK) return st;
   const float* qbar = pooled;
   const float* kbar = pooled + d.BH * d.nsb * d.D;
-  const unsigned tiles = (unsigned)((d.nsb + kTile - 1) / kTile);
-  dim3 sg(tiles, tiles, (unsigned)d.BH);
-  switch (d.r) {
-    case 1: score_kernel<1><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    case 2: score_kernel<2><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    case 4: score_kernel<4><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-    default: score_kernel<8><<<sg, 256, 0, cs>>>(qbar, kbar, scores, d.D, d.nsb, d.nb, scale); break;
-  }
-  return dfs::launch_status();
+  return launch_score(d, qbar, kbar, scores, scale, cs);
 }
