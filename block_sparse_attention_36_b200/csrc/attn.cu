@@ -9,7 +9,10 @@
 // one head, or rows order[2x], order[2x+1] of a work order), each with its
 // own kept list. While the softmax of one slot runs, the tensor pipe works
 // on the other slot's products, so neither the tensor pipe nor the
-// exponential units wait on each other for long.
+// exponential units wait on each other for long. The CTAs of a last,
+// partial wave may instead each take one query block and give each slot
+// half of its kept list; the two softmax warpgroups then merge their
+// (max, sum, O) in the epilogue, so that wave takes about half as long.
 // Warp roles (384 threads, three warpgroups):
 //   thread 0   initialises the barriers and starts the Q_A, Q_B loads at
 //              once (they depend only on the block index).
@@ -34,7 +37,9 @@
 //              (an older maximum stays exact as long as P and the row sum
 //              use the same one); epilogue normalises O_X and stores bf16
 //              rows (in curve order, or straight to raster order through
-//              perm) and the log-sum-exp.
+//              perm) and the log-sum-exp; in a split CTA slot B passes its
+//              (max, sum) through shared memory and slot A reads O_B from
+//              tensor memory and writes the merged rows.
 // Tensor memory: S_A | S_B | O_A | O_B (BLK, BLK, D, D fp32 columns).
 // Every mbarrier wait is bounded (DFS_FLAG_WAIT_TIMEOUT, early return);
 // copies and MMAs in flight are drained before tensor memory is released.
@@ -121,15 +126,23 @@ struct FrameMask {
   int P, T, T_per, s0, C, nG;
 };
 // Output rows go to op in curve order, or, when perm is set, straight to
-// their raster place o[b, perm[i], h, :] (o: [B, N, nh, D]). When order is
-// set, CTA c takes the query rows (b * nh + h) * nb + I at order[2c] and
-// order[2c + 1] (rows = B * nh * nb entries) instead of blocks 2c, 2c + 1
-// of head blockIdx.y.
+// their raster place o[b, perm[i], h, :] (o: [B, N, nh, D]).
+// Query rows are numbered by a virtual index v. With a work order, v is the
+// row (b * nh + h) * nb + I at order[v] (rows = B * nh * nb entries);
+// without one, v = 2 (bh * P + x) + e is block 2x + e of head bh, with
+// P = ceil(nb / 2) (block nb: an empty slot). CTA c < split_from takes rows
+// 2c and 2c + 1, one per slot. A CTA c >= split_from takes the one row
+// 2 split_from + (c - split_from) and gives each slot half of its kept list;
+// the epilogue merges the two partial softmax states. The host sets
+// split_from so that the last, partial wave of two-row CTAs becomes twice
+// as many half-length CTAs (tail_split) or leaves it at the CTA count.
 struct OutMap {
   const int32_t* perm;
   int nh;
   const int32_t* order;
   long long rows;
+  int tail_split;
+  long long split_from;
 };
 
 constexpr int kFrameRows = 3;
@@ -151,18 +164,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // (head, query block) of each slot; an empty slot gets block nb
-  int bh0 = blockIdx.y, bh1 = blockIdx.y, I0 = 2 * blockIdx.x, I1 = 2 * blockIdx.x + 1;
-  if (om.order) {
-    const long long pos = 2LL * blockIdx.x;
-    const int r0 = om.order[pos];
-    const int r1 = pos + 1 < om.rows ? om.order[pos + 1] : -1;
-    bh0 = r0 / nb;
-    I0 = r0 - bh0 * nb;
-    bh1 = r1 >= 0 ? r1 / nb : 0;
-    I1 = r1 >= 0 ? r1 - bh1 * nb : nb;
-  }
+  const long long cta = blockIdx.x;
+  const bool split = cta >= om.split_from;          // one row, half of its list per slot
+  const long long v0 = split ? 2 * om.split_from + (cta - om.split_from) : 2 * cta;
+  const long long v1 = split ? v0 : v0 + 1;
+  auto decode = [&](long long v, int& bh, int& I) {
+    if (om.order) {
+      const int r = v < om.rows ? om.order[v] : -1;
+      bh = r >= 0 ? r / nb : 0;
+      I = r >= 0 ? r - bh * nb : nb;
+    } else {
+      const long long P = (nb + 1) >> 1;
+      const long long p = v >> 1;
+      bh = (int)(p / P);
+      I = 2 * (int)(p - bh * P) + (int)(v & 1);
+    }
+  };
+  int bh0, I0, bh1, I1;
+  decode(v0, bh0, I0);
+  decode(v1, bh1, I1);
   auto slot_bh = [&](int x) { return x ? bh1 : bh0; };
-  auto slot_I = [&](int x) { return x ? I1 : I0; };   // frame-exact masking (no order): I1 = I0 + 1
+  // frame-exact masking (no order): I1 = I0 + 1, or I1 = I0 in a split CTA
+  auto slot_I = [&](int x) { return x ? I1 : I0; };
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
@@ -203,13 +226,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int J_first = lane < lim ? src[lane] : -1;    // fetched alongside the count
       int cnt = kv_cnt[row_id];
       cnt = max(0, min(cnt, lim));
+      // entries [lo, hi) of the row: all of it, or one half in a split CTA
+      int lo = 0, hi = cnt;
+      if (split) {
+        const int h0 = (cnt + 1) >> 1;
+        lo = x ? h0 : 0;
+        hi = x ? cnt : h0;
+      }
       int32_t* dst = lists + x * max_list;
-      for (int j0 = 0; j0 < cnt; j0 += 32) {
+      for (int j0 = lo; j0 < hi; j0 += 32) {
         const int j = j0 + lane;
         int J = -1;
-        if (j < cnt) J = (j0 == 0) ? J_first : src[j];
-        const bool ok = (j < cnt) && J >= 0 && J < nb;
-        bad |= (j < cnt) && !ok;
+        if (j < hi) J = (j0 == 0) ? J_first : src[j];
+        const bool ok = (j < hi) && J >= 0 && J < nb;
+        bad |= (j < hi) && !ok;
         const unsigned m = __ballot_sync(0xffffffffu, ok);
         if (ok) {
           const int pos = base + __popc(m & ((1u << lane) - 1u));
@@ -232,6 +262,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // FRAME only: per list entry (first key frame << 8 | columns in it), then the frame bit sets
   const int32_t* kmeta = lists + 2 * max_list;
   uint32_t* ftab = reinterpret_cast<uint32_t*>(lists + 4 * max_list);
+  // split CTAs: slot B's row maxima and sums for the merge (2 x 128 floats)
+  float* xch = reinterpret_cast<float*>(lists + (FRAME ? 4 * max_list + kFrameRows * frame_words(fm.T) : 2 * max_list));
   const int qf_lo = FRAME ? (I0 * BLK) / fm.P : 0;
   if (FRAME && warp >= 4) {
     const int words = frame_words(fm.T);
@@ -507,6 +539,74 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ---------------------------------------------------------- epilogue
     if (ok && nx > 0) ok = mbar_wait_bounded(&bars->o_final[x], 0, abort_flag, kWaitLimit);
     tc_fence_after();
+    if (split) {
+      // Both slots hold the same query rows over disjoint halves of the
+      // list: slot B hands its (m, l) to slot A, whose threads read O_B from
+      // tensor memory (same lane quarter) and write the merged rows.
+      if (x == 1) {
+        xch[r] = (nx > 0 && ok) ? m : -INFINITY;
+        xch[kQRows + r] = (nx > 0 && ok) ? l : 0.f;
+      }
+      tc_fence_before();
+      asm volatile("bar.sync 1, 256;" ::: "memory");   // the two softmax warpgroups
+      tc_fence_after();
+    }
+    if (split && n[1] > 0) {
+      if (x == 0) {
+        // O = (2^(m_A - M) O_A + 2^(m_B - M) O_B) / (2^(m_A - M) l_A + 2^(m_B - M) l_B),
+        // M = max(m_A, m_B); a half with no unmasked key has m = -inf and weight 0
+        const float mA = (nx > 0 && ok) ? m : -INFINITY, lA = (nx > 0 && ok) ? l : 0.f;
+        const float mB = xch[r], lB = xch[kQRows + r];
+        const float M = fmaxf(mA, mB);
+        const float aA = (mA == -INFINITY) ? 0.f : ex2(mA - M);
+        const float aB = (mB == -INFINITY) ? 0.f : ex2(mB - M);
+        const float L = lA * aA + lB * aB;
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+        const float wA = aA * inv, wB = aB * inv;
+        const long long qrow = (long long)I * BLK + r;
+        const bool store = ok && I < nb && r < BLK && qrow < N;
+        __nv_bfloat16* orow;
+        if (om.perm) {
+          const int b = bh / om.nh, h = bh - b * om.nh;
+          const long long tok = (qrow < N) ? om.perm[qrow] : 0;
+          orow = op + (((long long)b * N + tok) * om.nh + h) * D;
+        } else {
+          orow = op + ((long long)bh * N + qrow) * D;
+        }
+        const uint32_t oB_addr = tmem + lane_base + C::o_col(1);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ra[32], rb[32];
+          if (nx > 0) {
+            tmem_ld32(o_addr + c * 32, ra);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ra[e] = 0u;
+          }
+          tmem_ld32(oB_addr + c * 32, rb);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              float t = 0.f;
+              if (wA != 0.f) t = __uint_as_float(ra[2 * e + u]) * wA;
+              if (wB != 0.f) t = fmaf(__uint_as_float(rb[2 * e + u]), wB, t);
+              v[u] = t;
+            }
+            pk[e] = pack_bf16x2(v[0], v[1]);
+          }
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+        if (store && lse) lse[(long long)bh * N + qrow] = (M + __log2f(L)) * 0.6931471805599453f;
+      }
+    } else if (!split || x == 0) {
     const long long qrow = (long long)I * BLK + r;
     const bool store = ok && I < nb && r < BLK && qrow < N;
     __nv_bfloat16* orow;
@@ -542,6 +642,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // natural-log LSE of the scaled logits: (m + log2 l) * ln 2
       lse[(long long)bh * N + qrow] = (nx > 0) ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
+    }
   }
 
   tc_fence_before();
@@ -562,7 +663,8 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
       !dfs::make_map_bf16(&mv, vp, d.N, D, d.BH, BLK))
     return DFS_ERR_CUDA;
   const int max_list = min(kcap, d.nb);
-  size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + 2 * (size_t)max_list * sizeof(int32_t);
+  size_t smem = 1024 + C::kBarOff + sizeof(Barriers) + 2 * (size_t)max_list * sizeof(int32_t) +
+                2 * kQRows * sizeof(float);
   if (FRAME) smem += 2 * (size_t)max_list * sizeof(int32_t) + (size_t)kFrameRows * frame_words(fm.T) * sizeof(uint32_t);
   if (smem > 232448) return DFS_ERR_UNSUPPORTED;
   // Tensor memory per SM is 512 columns: a 512-column CTA must be alone on
@@ -573,7 +675,25 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, EMU, FRAME>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return DFS_ERR_CUDA;
-  const dim3 grid = om.order ? dim3((unsigned)((d.BH * d.nb + 1) / 2), 1u) : dim3((unsigned)((d.nb + 1) / 2), (unsigned)d.BH);
+  // virtual rows (see OutMap), two-row CTAs, and the split of the last wave
+  const long long V = om.order ? om.rows : 2LL * d.BH * ((d.nb + 1) / 2);
+  const long long pairs = (V + 1) / 2;
+  om.split_from = pairs;
+  if (om.tail_split) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) {
+      // a last wave of rem two-row CTAs (rem <= SMs / 2) becomes 2 rem
+      // CTAs of half the work each, which all run at once
+      const long long rem = pairs % sms;
+      if (rem > 0 && 2 * rem <= sms) om.split_from = pairs - rem;
+    }
+  }
+  // two-row CTAs, plus one CTA per row after them (the last pair may hold
+  // one row when V is odd; it is split only together with its wave)
+  const long long ctas = om.split_from == pairs ? pairs : om.split_from + (V - 2 * om.split_from);
+  if (ctas > 0x7fffffffLL) return DFS_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)ctas);
   const float scale_log2 = scale * 1.4426950408889634f;
   attn_fwd_kernel<D, BLK, EMU, FRAME><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, kv_idx, kv_cnt, kcap, (int)d.N, d.nb, scale_log2, (__nv_bfloat16*)op, lse, max_list, fm, om);
@@ -622,7 +742,7 @@ extern "C" int dfs_sparse_attn_fwd(const dfs_shape* shape, const void* qp, const
   if (st != DFS_OK) return st;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
   return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream,
-                              FrameMask{1, 1, 1, 0, 1, 0}, OutMap{nullptr, 1, nullptr, 0});
+                              FrameMask{1, 1, 1, 0, 1, 0}, OutMap{nullptr, 1, nullptr, d.BH * d.nb, 1, 0});
 }
 
 extern "C" int dfs_sparse_attn_fwd_ex(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
@@ -632,12 +752,12 @@ extern "C" int dfs_sparse_attn_fwd_ex(const dfs_shape* shape, const void* qp, co
   const int st = check_attn_args(shape, qp, kp, vp, kv_idx, kv_cnt, kcap, o, lse, &d);
   if (st != DFS_OK) return st;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
-  OutMap om{nullptr, d.nh, nullptr, d.BH * d.nb};
+  OutMap om{nullptr, d.nh, nullptr, d.BH * d.nb, 1, 0};
   if (opts) {
     om.perm = opts->perm;
     om.order = opts->order;
+    om.tail_split = opts->no_tail_split ? 0 : 1;
   }
-  if (om.order && (d.BH * d.nb + 1) / 2 > 0x7fffffffLL) return DFS_ERR_UNSUPPORTED;
   return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse, (cudaStream_t)stream,
                               FrameMask{1, 1, 1, 0, 1, 0}, om);
 }
@@ -660,7 +780,7 @@ extern "C" int dfs_sparse_attn_lvsa_fwd(const dfs_shape* shape, const void* qp, 
   fm.C = lvsa->lvsa_C;
   fm.nG = (fm.s0 < d.T) ? (d.T - 1 - fm.s0) / fm.T_per + 1 : 0;
   return dispatch_attn<true>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream, fm,
-                             OutMap{nullptr, 1, nullptr, 0});
+                             OutMap{nullptr, 1, nullptr, d.BH * d.nb, 1, 0});
 }
 
 namespace {

@@ -59,7 +59,7 @@ class _Shape(ctypes.Structure):
 
 
 class _AttnOpts(ctypes.Structure):
-    _fields_ = [("perm", ctypes.c_void_p), ("order", ctypes.c_void_p)]
+    _fields_ = [("perm", ctypes.c_void_p), ("order", ctypes.c_void_p), ("no_tail_split", ctypes.c_int)]
 
 
 class _SelectParams(ctypes.Structure):
@@ -221,9 +221,10 @@ def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o
 
 
 def dfs_sparse_attn_fwd_ex(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse=None, perm=None,
-                           order=None, stream=None):
+                           order=None, stream=None, tail_split=True):
     sh = shape.c()
-    opts = _AttnOpts(None if perm is None else perm.data_ptr(), None if order is None else order.data_ptr())
+    opts = _AttnOpts(None if perm is None else perm.data_ptr(), None if order is None else order.data_ptr(),
+                     0 if tail_split else 1)
     _check("dfs_sparse_attn_fwd_ex", LIB.dfs_sparse_attn_fwd_ex(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
         ctypes.byref(opts), _ptr(o), _ptr(lse), _stream(stream)))

@@ -226,7 +226,7 @@ int dfs_sparse_attn_fwd(const dfs_shape *shape, const void *qp, const void *kp, 
                         const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
                         void *op, float *lse, dfs_stream_t stream);
 
-/* Options of dfs_sparse_attn_fwd_ex (NULL members: the defaults). */
+/* Options of dfs_sparse_attn_fwd_ex (zero / NULL members: the defaults). */
 typedef struct {
   /* perm (int32 [N], device; the index of dfs_hilbert_perm): write the row
    * of curve position i straight to its raster place o[b, perm[i], h, :],
@@ -235,10 +235,18 @@ typedef struct {
   const int32_t *perm;
   /* order (int32 [B * nh * nb], device; a permutation of the query rows
    * (b * nh + h) * nb + I, e.g. from dfs_attn_order): CTA c computes rows
-   * order[2c] and order[2c + 1]. Only the scheduling changes; every row's
-   * result is bitwise the same. NULL: CTA (x, b * nh + h) takes blocks
-   * 2x, 2x + 1 of that head.                                              */
+   * order[2c] and order[2c + 1]. Only the scheduling changes; with
+   * no_tail_split set, every row's result is bitwise that of the default
+   * order. NULL: CTAs take blocks 2x, 2x + 1 of one head, head by head.  */
   const int32_t *order;
+  /* no_tail_split: 0 (default) lets the launch turn its last, partial wave
+   * of two-row CTAs (when it holds at most half as many CTAs as the GPU
+   * has SMs) into one-row CTAs that give each half of the row's kept list
+   * to one of their two tiles and merge the two partial softmax states --
+   * the same rows in about half the time. The merged rows differ from the
+   * unsplit ones by rounding only. Nonzero: every CTA takes two rows.
+   * dfs_sparse_attn_fwd and dfs_sparse_attn_lvsa_fwd use the default.      */
+  int no_tail_split;
 } dfs_attn_opts;
 
 /* dfs_sparse_attn_fwd_ex -- dfs_sparse_attn_fwd with the options above.

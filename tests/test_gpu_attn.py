@@ -172,8 +172,8 @@ def test_scatter_epilogue_equals_fwd_then_unperm(lib, grid, D):
 @pytest.mark.parametrize("B,nh,D,N,kcap", [(1, 3, 128, 5000, 20), (2, 2, 64, 3000, 24)])
 def test_work_order_changes_nothing(lib, B, nh, D, N, kcap):
     """Rows run in count order (dfs_attn_order, dfs_attn_opts.order) give
-    bit for bit the rows of the default order; the order is a permutation
-    sorted by kept count, largest first."""
+    bit for bit the rows of the default order (tail split off); the order is
+    a permutation sorted by kept count, largest first."""
     blk = 128
     nb = -(-N // blk)
     rng = np.random.default_rng(B * N)
@@ -187,8 +187,10 @@ def test_work_order_changes_nothing(lib, B, nh, D, N, kcap):
     a, b = torch.empty_like(qp), torch.empty_like(qp)
     la = torch.empty((B, nh, N), dtype=torch.float32, device="cuda")
     lb = torch.empty_like(la)
-    lib.dfs_sparse_attn_fwd(s, qp, kp, vp, it, ct, kcap, 0.0, a, la)
-    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, b, lb, order=order)
+    # every CTA on two rows in both launches (a split tail would merge
+    # different rows in the two orders)
+    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, a, la, tail_split=False)
+    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, b, lb, order=order, tail_split=False)
     torch.cuda.synchronize()
     o = order.cpu().numpy()
     assert np.array_equal(np.sort(o), np.arange(B * nh * nb))
@@ -196,3 +198,81 @@ def test_work_order_changes_nothing(lib, B, nh, D, N, kcap):
     assert (np.diff(counts) <= 0).all()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert torch.equal(la, lb)
+
+
+@pytest.mark.parametrize("nh,D,N,kcap,with_order", [(5, 128, 8192, 9, False), (3, 64, 14158, 7, True)])
+def test_tail_split(lib, nh, D, N, kcap, with_order):
+    """The last, partial wave of two-row CTAs runs as one-row CTAs whose two
+    tiles take one half of the row's list each and merge (m, l, O): those
+    rows match the oracle and the unsplit launch up to rounding, every other
+    row is bitwise the unsplit one. The split rows include lists of 0, 1, 2
+    and 3 entries, an invalid entry that empties the first half, and (with a
+    work order) an odd number of rows."""
+    blk, B = 128, 1
+    nb = -(-N // blk)
+    rng = np.random.default_rng(N + nh)
+    idx = np.full((B, nh, nb, kcap), -1, dtype=np.int32)
+    cnt = np.zeros((B, nh, nb), dtype=np.int32)
+    for h in range(nh):
+        for I in range(nb):
+            c = kcap if I < nb - 4 or h < nh - 1 else I - (nb - 4)      # last rows of the last head: 0, 1, 2, 3
+            idx[0, h, I, :c] = np.sort(rng.choice(nb, size=c, replace=False))
+            cnt[0, h, I] = c
+    ref_idx, ref_cnt = idx.copy(), cnt.copy()
+    idx[0, nh - 1, nb - 2, 0] = nb + 5          # the 2-entry row: its first half holds only this
+    ref_idx[0, nh - 1, nb - 2, :2] = [idx[0, nh - 1, nb - 2, 1], -1]
+    ref_cnt[0, nh - 1, nb - 2] = 1
+    g = torch.Generator().manual_seed(N)
+    q, k, v = (torch.randn((B, nh, N, D), generator=g).to(torch.bfloat16) for _ in range(3))
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, 16)
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    order = None
+    if with_order:
+        order = torch.empty(B * nh * nb, dtype=torch.int32, device="cuda")
+        lib.dfs_attn_order(s, ct, kcap, order)
+    outs = []
+    for split in (True, False):
+        o = torch.empty((B, nh, N, D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B, nh, N), dtype=torch.float32, device="cuda")
+        lib.dfs_sparse_attn_fwd_ex(s, q.cuda(), k.cuda(), v.cuda(), it, ct, kcap, 0.0, o, lse, order=order,
+                                   tail_split=split)
+        outs.append((o, lse))
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == lib.DFS_FLAG_BAD_KV_INDEX
+    # the rows of the split CTAs, from the launch geometry
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    V = B * nh * nb if with_order else 2 * B * nh * ((nb + 1) // 2)
+    pairs = (V + 1) // 2
+    rem = pairs % sms
+    assert 0 < rem and 2 * rem <= sms, "the case must have a split tail"
+    split_rows = np.zeros((B * nh, nb), dtype=bool)
+    rows = order.cpu().numpy() if with_order else None
+    for vr in range(2 * (pairs - rem), V):
+        if with_order:
+            r = int(rows[vr])
+            split_rows[r // nb, r % nb] = True
+        else:
+            p, e = divmod(vr, 2)
+            bh, x = divmod(p, (nb + 1) // 2)
+            if 2 * x + e < nb:
+                split_rows[bh, 2 * x + e] = True
+    assert split_rows[nh - 1, nb - 4:].all()
+    tok = np.repeat(split_rows, blk, axis=1)[:, :N].reshape(B, nh, N)
+    a, b = (x[0].float().cpu().numpy() for x in outs)
+    la, lb = (x[1].cpu().numpy() for x in outs)
+    ref, rlse = attention.block_sparse_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                                 ref_idx, ref_cnt, blk)
+
+    def where(mask):
+        pos = np.argwhere(mask.reshape(B * nh, N))[:6]
+        return [(int(h), int(t) // blk, int(t), float(la.reshape(-1, N)[h, t]), float(lb.reshape(-1, N)[h, t]),
+                 float(rlse.reshape(-1, N)[h, t]), int(cnt.reshape(-1, nb)[h, t // blk])) for h, t in pos]
+
+    rf = np.isfinite(rlse)
+    assert np.array_equal(rf, np.isfinite(lb)), where(rf != np.isfinite(lb))
+    assert np.array_equal(rf, np.isfinite(la)), where(rf != np.isfinite(la))
+    assert np.abs(la[rf] - rlse[rf]).max() < 1e-3
+    assert_attn_close(a, ref, "tail-split output")
+    assert np.array_equal(a[~tok], b[~tok]) and np.array_equal(la[~tok], lb[~tok])
+    assert np.abs(la[tok & rf] - lb[tok & rf]).max() < 1e-4
+    assert np.abs(a[tok] - b[tok]).max() <= 2 ** -7 * max(1.0, np.abs(b[tok]).max())
