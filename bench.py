@@ -50,7 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch from one ncu capture
 # (profiles/attn_fwd_<workload>.md), valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
-ATTN_TRAFFIC = {"wan_1p3b_layer": (298_804_224 + 82_775_296, "c065d4b64fbb38ab")}
+ATTN_TRAFFIC = {"wan_1p3b_layer": (298_958_592 + 83_133_184, "95155120f61bbb8a")}
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 
