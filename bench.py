@@ -56,7 +56,7 @@ ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa
 
 # dram read + write of one backward call (all its launches) on the Wan layer,
 # from a one-pass ncu capture of these sources
-BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_195_136 + 263_207_424, "52bad2f1fdf8b4eb")}
+BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_816_448 + 262_639_360, "a64bc91715fa78dd")}
 BWD_SOURCES = ("attn_bwd.cu", "sm100_ptx.cuh", "common.cuh", "tmap.cuh")
 
 
