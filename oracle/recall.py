@@ -12,8 +12,11 @@ synthetic workload at the same keep budget:
 
     python -m oracle.recall --workload wan_1p3b_layer --queries 256
 
-Parity unpinned: there is nothing to compare the values with; only their
-ordering across variants is read.
+Pinned by closed forms (tests/test_oracle_attention.py): every block kept
+gives 1, none kept gives 0, and a one-block mask gives the kept softmax mass
+computed by brute force. There is no GPU counterpart to compare with: the
+diagnostic only ranks orders and scoring granularities, and the pages print
+no recall values to compare its numbers with.
 """
 from __future__ import annotations
 
