@@ -1,9 +1,12 @@
 """GPU pooling and hierarchical block scores against the fp64 oracle.
 
 Page: DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
-Generation, Methodology item 2. The GPU computes in fp32; the bound used
-here is the fp32 rounding of sums of <= sb bf16 values and of D-term dot
-products (relative error ~ (D + sb) * 2^-24 of the magnitudes summed)."""
+Generation, Methodology item 2. The means are fp32 sums of <= sb bf16
+values; the dot products run on the tensor cores as three tf32 products of
+split operands (x = x_hi + x_lo, both tf32-rounded), each term within
+3 * 2^-22 = 12 u of |a||b| (u = 2^-24), accumulated in fp32 over
+3 * D / 8 MMA steps. Both fit the bound used here, (D + 2 sb + 4) u times
+the magnitudes summed: 12 + 3 D / 8 <= D for D >= 64."""
 import math
 
 import numpy as np
