@@ -633,7 +633,10 @@ def run_reference(args):
     qkv = synth.workload_inputs(wl, seed=args.seed)
     k = wl.ratio_count(wl.keep_num) if wl.mode == "topk" else 0
     cap = wl.ratio_count(wl.cap_num) if wl.mode == "threshold" else 0
-    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    # seconds of oracle work per timed step (warm-up steps a quarter of it):
+    # 2 to 20 s so that the whole run stays within a few minutes, and never
+    # more than --cpu-seconds
+    budget = max(min(2.0, args.cpu_seconds), min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(wl, qkv, k, cap, budget_s=budget / 4)
     vals = [cpu_baseline(wl, qkv, k, cap, budget_s=budget) for _ in range(args.steps)]
