@@ -47,8 +47,8 @@ METRIC = "block-sparse attn ms/call & kept-block TFLOP/s vs B200 bf16 TC peak"
 KERNELS_PER_STEP = {"topk": 4, "threshold": 5, "global": 5, "lvsa": 5, "radial": 5}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per attention launch from one ncu capture
-# (profiles/attn_fwd_<workload>.md), valid only for the attention sources
+# DRAM bytes (read + write) per attention launch from one ncu capture of
+# that workload, valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
 ATTN_TRAFFIC = {"wan_1p3b_layer": (298_958_592 + 83_133_184, "95155120f61bbb8a")}
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")

@@ -105,14 +105,52 @@ LIB = _load()
 
 
 class DfsError(RuntimeError):
-    def __init__(self, call, status):
-        super().__init__(f"{call}: {LIB.dfs_status_string(status).decode()} ({status})")
+    def __init__(self, call, status, detail=None):
+        msg = f"{call}: {LIB.dfs_status_string(status).decode()} ({status})"
+        super().__init__(msg if detail is None else f"{msg}: {detail}")
         self.status = status
 
 
 def _check(call, status):
     if status != DFS_OK:
         raise DfsError(call, status)
+
+
+def _need(call, name, t, numel, dtype, optional=False):
+    """Host check of one tensor argument before its pointer goes to C: a CUDA
+    tensor of the expected dtype, contiguous, holding at least ``numel``
+    elements (the size the shape implies). The C side cannot see sizes, so a
+    wrong tensor would otherwise become an out-of-bounds device access."""
+    if t is None:
+        if optional:
+            return
+        raise DfsError(call, DFS_ERR_INVALID_ARG, f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise DfsError(call, DFS_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise DfsError(call, DFS_ERR_INVALID_ARG, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise DfsError(call, DFS_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise DfsError(call, DFS_ERR_INVALID_ARG, f"{name} holds {t.numel()} elements, the shape needs {numel}")
+
+
+def _need_ws(call, ws):
+    """A workspace may have any dtype (its size in bytes is checked by the C
+    side), but it must be contiguous device memory."""
+    if ws is not None and (not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous()):
+        raise DfsError(call, DFS_ERR_INVALID_ARG, "ws must be a contiguous CUDA tensor")
+
+
+_BF16, _F32, _I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def _tok(shape):      # elements of one [B, N, nh, D] / [B, nh, N, D] tensor
+    return shape.B * shape.nh * shape.N * shape.D
+
+
+def _rows(shape):     # query rows (b, h, I)
+    return shape.B * shape.nh * shape.nb
 
 
 @dataclass(frozen=True)
@@ -146,6 +184,10 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -154,6 +196,11 @@ def _stream(stream):
 
 def dfs_hilbert_perm(shape: Shape, order, perm, inv, build_index, q, k, v, qp, kp, vp, stream=None):
     order = ORDERS.get(order, order)
+    c = "dfs_hilbert_perm"
+    _need(c, "perm", perm, shape.N, _I32)
+    _need(c, "inv", inv, shape.N, _I32, optional=not build_index)
+    for n, t in (("q", q), ("k", k), ("v", v), ("qp", qp), ("kp", kp), ("vp", vp)):
+        _need(c, n, t, _tok(shape), _BF16, optional=True)
     sh = shape.c()
     _check("dfs_hilbert_perm", LIB.dfs_hilbert_perm(
         ctypes.byref(sh), int(order), _ptr(perm), _ptr(inv), int(bool(build_index)),
@@ -162,17 +209,27 @@ def dfs_hilbert_perm(shape: Shape, order, perm, inv, build_index, q, k, v, qp, k
 
 def dfs_hilbert_perm_pooled(shape: Shape, order, perm, inv, build_index, q, k, v, qp, kp, vp, ws, stream=None):
     order = ORDERS.get(order, order)
+    c = "dfs_hilbert_perm_pooled"
+    _need(c, "perm", perm, shape.N, _I32)
+    _need(c, "inv", inv, shape.N, _I32, optional=not build_index)
+    for n, t in (("q", q), ("k", k), ("qp", qp), ("kp", kp)):
+        _need(c, n, t, _tok(shape), _BF16)
+    for n, t in (("v", v), ("vp", vp)):
+        _need(c, n, t, _tok(shape), _BF16, optional=True)
+    _need_ws(c, ws)
     sh = shape.c()
     _check("dfs_hilbert_perm_pooled", LIB.dfs_hilbert_perm_pooled(
         ctypes.byref(sh), int(order), _ptr(perm), _ptr(inv), int(bool(build_index)),
-        _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(ws), ws.numel() * ws.element_size(),
+        _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(ws), _nbytes(ws),
         _stream(stream)))
 
 
 def dfs_block_score_pooled(shape: Shape, scale, scores, ws, stream=None):
+    _need("dfs_block_score_pooled", "scores", scores, _rows(shape) * shape.nb, _F32)
+    _need_ws("dfs_block_score_pooled", ws)
     sh = shape.c()
     _check("dfs_block_score_pooled", LIB.dfs_block_score_pooled(
-        ctypes.byref(sh), float(scale), _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(),
+        ctypes.byref(sh), float(scale), _ptr(scores), _ptr(ws), _nbytes(ws),
         _stream(stream)))
 
 
@@ -182,6 +239,10 @@ def dfs_workspace_bytes(shape: Shape, which=DFS_WS_BLOCK_SCORE) -> int:
 
 
 def dfs_block_score(shape: Shape, qp, kp, scale, scores, ws, stream=None):
+    for n, t in (("qp", qp), ("kp", kp)):
+        _need("dfs_block_score", n, t, _tok(shape), _BF16)
+    _need("dfs_block_score", "scores", scores, _rows(shape) * shape.nb, _F32)
+    _need_ws("dfs_block_score", ws)
     sh = shape.c()
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("dfs_block_score", LIB.dfs_block_score(
@@ -192,6 +253,9 @@ def dfs_block_score_noalloc(shape: Shape, qp, kp, scale, scores, stream=None):
     """dfs_block_score with the library's built-in scratch buffer instead of a
     workspace, for callers that cannot allocate device memory (see the C
     header for the size limit, first-call set-up and the sharing rule)."""
+    for n, t in (("qp", qp), ("kp", kp)):
+        _need("dfs_block_score_noalloc", n, t, _tok(shape), _BF16)
+    _need("dfs_block_score_noalloc", "scores", scores, _rows(shape) * shape.nb, _F32)
     sh = shape.c()
     _check("dfs_block_score_noalloc", LIB.dfs_block_score_noalloc(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), float(scale), _ptr(scores), _stream(stream)))
@@ -207,13 +271,27 @@ def select_params(mode, k=0, cap=0, tau=0.0, lvsa_T_per=8, lvsa_C=21, lvsa_step=
 
 
 def dfs_select_mask(shape: Shape, scores, params, kv_idx, kv_cnt, kcap, stream=None):
+    c = "dfs_select_mask"
+    _need(c, "scores", scores, _rows(shape) * shape.nb, _F32,
+          optional=params.mode in (DFS_SEL_LVSA, DFS_SEL_RADIAL))
+    _need(c, "kv_idx", kv_idx, _rows(shape) * max(1, int(kcap)), _I32)
+    _need(c, "kv_cnt", kv_cnt, _rows(shape), _I32)
     sh = shape.c()
     _check("dfs_select_mask", LIB.dfs_select_mask(
         ctypes.byref(sh), _ptr(scores), ctypes.byref(params), _ptr(kv_idx), _ptr(kv_cnt), int(kcap),
         _stream(stream)))
 
 
+def _need_attn(c, shape, qp, kp, vp, kv_idx, kv_cnt, kcap, o, lse):
+    for n, t in (("qp", qp), ("kp", kp), ("vp", vp), ("o", o)):
+        _need(c, n, t, _tok(shape), _BF16)
+    _need(c, "kv_idx", kv_idx, _rows(shape) * max(1, int(kcap)), _I32)
+    _need(c, "kv_cnt", kv_cnt, _rows(shape), _I32)
+    _need(c, "lse", lse, shape.B * shape.nh * shape.N, _F32, optional=True)
+
+
 def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse=None, stream=None):
+    _need_attn("dfs_sparse_attn_fwd", shape, qp, kp, vp, kv_idx, kv_cnt, kcap, op, lse)
     sh = shape.c()
     _check("dfs_sparse_attn_fwd", LIB.dfs_sparse_attn_fwd(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
@@ -222,6 +300,10 @@ def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o
 
 def dfs_sparse_attn_fwd_ex(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse=None, perm=None,
                            order=None, stream=None, tail_split=True):
+    c = "dfs_sparse_attn_fwd_ex"
+    _need_attn(c, shape, qp, kp, vp, kv_idx, kv_cnt, kcap, o, lse)
+    _need(c, "perm", perm, shape.N, _I32, optional=True)
+    _need(c, "order", order, _rows(shape), _I32, optional=True)
     sh = shape.c()
     opts = _AttnOpts(None if perm is None else perm.data_ptr(), None if order is None else order.data_ptr(),
                      0 if tail_split else 1)
@@ -231,6 +313,8 @@ def dfs_sparse_attn_fwd_ex(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale
 
 
 def dfs_attn_order(shape: Shape, kv_cnt, kcap, order, stream=None):
+    _need("dfs_attn_order", "kv_cnt", kv_cnt, _rows(shape), _I32)
+    _need("dfs_attn_order", "order", order, _rows(shape), _I32)
     sh = shape.c()
     _check("dfs_attn_order", LIB.dfs_attn_order(ctypes.byref(sh), _ptr(kv_cnt), int(kcap), _ptr(order),
                                                 _stream(stream)))
@@ -238,6 +322,14 @@ def dfs_attn_order(shape: Shape, kv_cnt, kcap, order, stream=None):
 
 def dfs_sparse_attn_bwd(shape: Shape, qp, kp, vp, op, dop, lse, kv_idx, kv_cnt, kcap, scale, dqp, dkp, dvp, ws,
                         stream=None):
+    c = "dfs_sparse_attn_bwd"
+    for n, t in (("qp", qp), ("kp", kp), ("vp", vp), ("op", op), ("dop", dop), ("dqp", dqp), ("dkp", dkp),
+                 ("dvp", dvp)):
+        _need(c, n, t, _tok(shape), _BF16)
+    _need(c, "lse", lse, shape.B * shape.nh * shape.N, _F32)
+    _need(c, "kv_idx", kv_idx, _rows(shape) * max(1, int(kcap)), _I32)
+    _need(c, "kv_cnt", kv_cnt, _rows(shape), _I32)
+    _need_ws(c, ws)
     sh = shape.c()
     _check("dfs_sparse_attn_bwd", LIB.dfs_sparse_attn_bwd(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(op), _ptr(dop), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt),
@@ -247,6 +339,7 @@ def dfs_sparse_attn_bwd(shape: Shape, qp, kp, vp, op, dop, lse, kv_idx, kv_cnt, 
 
 def dfs_sparse_attn_lvsa_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, params, op, lse=None,
                              stream=None):
+    _need_attn("dfs_sparse_attn_lvsa_fwd", shape, qp, kp, vp, kv_idx, kv_cnt, kcap, op, lse)
     sh = shape.c()
     _check("dfs_sparse_attn_lvsa_fwd", LIB.dfs_sparse_attn_lvsa_fwd(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
@@ -254,6 +347,9 @@ def dfs_sparse_attn_lvsa_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, sca
 
 
 def dfs_unperm(shape: Shape, perm, op, o, stream=None):
+    _need("dfs_unperm", "perm", perm, shape.N, _I32)
+    _need("dfs_unperm", "op", op, _tok(shape), _BF16)
+    _need("dfs_unperm", "o", o, _tok(shape), _BF16)
     sh = shape.c()
     _check("dfs_unperm", LIB.dfs_unperm(ctypes.byref(sh), _ptr(perm), _ptr(op), _ptr(o), _stream(stream)))
 

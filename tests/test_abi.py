@@ -128,3 +128,35 @@ def test_argument_errors_of_later_entry_points(lib):
     assert L.dfs_select_mask(ctypes.byref(sh), None, ctypes.byref(prm), fake, fake, 8, None) == -1
     big = _shape_c(lib, B=8, nh=16, T=64, H=64, W=64, blk=128, sb=32)   # pooled means >> 32 MiB
     assert L.dfs_block_score_noalloc(ctypes.byref(big), fake, fake, 0.0, fake, None) == -6
+
+
+def test_noalloc_limit_matches_the_header(lib):
+    """The binding's copy of the built-in scratch size is the header's."""
+    txt = open(HEADER).read()
+    m = re.search(r"#define\s+DFS_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", txt)
+    assert m, "DFS_NOALLOC_SCRATCH_BYTES not found"
+    assert lib.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_binding_rejects_host_tensors_before_calling_c(lib):
+    """The wrappers check tensor arguments on the host: a CPU tensor or a
+    missing required tensor raises DfsError(DFS_ERR_INVALID_ARG) without
+    reaching the library (so no device pointer is ever formed from it)."""
+    import torch
+    s = lib.Shape(1, 2, 64, 8, 16, 16, 64, 16)
+    x = torch.zeros((1, s.N, 2, 64), dtype=torch.bfloat16)
+    scores = torch.zeros((1, 2, s.nb, s.nb), dtype=torch.float32)
+    idx = torch.zeros((1, 2, s.nb, 8), dtype=torch.int32)
+    cnt = torch.zeros((1, 2, s.nb), dtype=torch.int32)
+    calls = [
+        lambda: lib.dfs_block_score(s, x, x, 0.0, scores, None),
+        lambda: lib.dfs_block_score_noalloc(s, x, x, 0.0, scores),
+        lambda: lib.dfs_select_mask(s, scores, lib.select_params("topk", k=8), idx, cnt, 8),
+        lambda: lib.dfs_sparse_attn_fwd(s, x, x, x, idx, cnt, 8, 0.0, x),
+        lambda: lib.dfs_unperm(s, None, x, x),
+        lambda: lib.dfs_attn_order(s, cnt, 8, cnt),
+    ]
+    for call in calls:
+        with pytest.raises(lib.DfsError) as e:
+            call()
+        assert e.value.status == lib.DFS_ERR_INVALID_ARG

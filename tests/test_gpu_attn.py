@@ -276,3 +276,31 @@ def test_tail_split(lib, nh, D, N, kcap, with_order):
     assert np.array_equal(a[~tok], b[~tok]) and np.array_equal(la[~tok], lb[~tok])
     assert np.abs(la[tok & rf] - lb[tok & rf]).max() < 1e-4
     assert np.abs(a[tok] - b[tok]).max() <= 2 ** -7 * max(1.0, np.abs(b[tok]).max())
+
+
+def test_binding_rejects_wrong_tensors(lib):
+    """The wrappers check device, dtype, contiguity and size against the
+    shape before any pointer reaches the library; a rejected call launches
+    nothing (the output keeps its contents)."""
+    B, nh, D, blk, N = 1, 2, 64, 64, 512
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, 16)
+    q = torch.zeros((B, nh, N, D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((B, nh, s.nb, 2), dtype=torch.int32, device="cuda")
+    cnt = torch.ones((B, nh, s.nb), dtype=torch.int32, device="cuda")
+    op = torch.full((B, nh, N, D), 7.0, dtype=torch.bfloat16, device="cuda")
+    bad = [
+        dict(q=q[:, :, : N // 2].contiguous()),                   # too small for the shape
+        dict(q=q.float()),                                        # wrong dtype
+        dict(q=q.transpose(2, 3)),                                # not contiguous
+        dict(idx=idx[..., :1].contiguous()),                      # kv_idx shorter than kcap
+        dict(cnt=cnt.to(torch.int64)),
+        dict(op=op[:, :1].contiguous()),
+    ]
+    for case in bad:
+        a = dict(q=q, idx=idx, cnt=cnt, op=op)
+        a.update(case)
+        with pytest.raises(lib.DfsError) as e:
+            lib.dfs_sparse_attn_fwd(s, a["q"], q, q, a["idx"], a["cnt"], 2, 0.0, a["op"])
+        assert e.value.status == lib.DFS_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert bool((op == 7.0).all())

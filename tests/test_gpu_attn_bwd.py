@@ -145,7 +145,11 @@ def test_rejects_blk64_and_short_workspace(lib):
     lse = torch.zeros((1, 1, 256), dtype=torch.float32, device="cuda")
     idx = torch.zeros((1, 1, 2, 1), dtype=torch.int32, device="cuda")
     cnt = torch.ones((1, 1, 2), dtype=torch.int32, device="cuda")
-    small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    # a short view of a buffer large enough for the call: a size check that
+    # failed to reject it would still write only memory this test owns
+    need = lib.dfs_workspace_bytes(s, lib.DFS_WS_ATTN_BWD)
+    big = torch.empty(need, dtype=torch.uint8, device="cuda")
+    small = big[:256]
     with pytest.raises(RuntimeError, match="workspace"):
         lib.dfs_sparse_attn_bwd(s, x, x, x, x, x, lse, idx, cnt, 1, 0.0, x, x, x, small)
     with pytest.raises(RuntimeError, match="unsupported"):
