@@ -480,11 +480,19 @@ def run_backward(args):
         dist.destroy_process_group()
 
 
+def schedule_config(wl):
+    return (f"{wl.name}: B={wl.B} nh={wl.nh} D={wl.D} grid {wl.T}x{wl.H}x{wl.W} (N={wl.N}) {wl.order} order, "
+            f"blk {wl.blk}, sb {wl.sb}, {wl.n_steps} steps, top-k 103 -> 32 of {wl.nb}, "
+            f"mask refresh every {wl.refresh} steps, attention every step")
+
+
 def run_schedule(args, wl, rank, world, local):
     """The 50-step denoising loop: Q/K change every step (V is fixed), the
     keep budget falls from 40 % to 10 %, masks are rebuilt every 5 steps and
     attention runs every step. Reports the amortised time per step and the
-    kept-block TFLOP/s over all 50 steps."""
+    kept-block TFLOP/s over all 50 steps; the roofline object reports the
+    attention kernel over the loop, e2e the loop through the public API from
+    pinned host buffers."""
     import torch
     import synth
     import block_sparse_attention_36_b200 as bsa
@@ -492,33 +500,40 @@ def run_schedule(args, wl, rank, world, local):
     from block_sparse_attention_36_b200 import schedule
 
     s = bsa.Shape(wl.B, wl.nh, wl.D, wl.T, wl.H, wl.W, wl.blk, wl.sb)
-    kmax = schedule.keep_budget(0, s.nb, wl.n_steps, wl.refresh)
-    layer = bsa.DfsLayer(s, order=wl.order, mode="topk", k=kmax, kcap=kmax)
+    ks = [schedule.keep_budget(st, s.nb, wl.n_steps, wl.refresh) for st in range(wl.n_steps)]
+    refresh = [schedule.is_refresh(st, wl.refresh) for st in range(wl.n_steps)]
+    layer = bsa.DfsLayer(s, order=wl.order, mode="topk", k=ks[0], kcap=ks[0])
     fields = {n: t.cuda() for n, t in synth.schedule_fields(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=args.seed + rank).items()}
     v = synth.field_qkv(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=args.seed + rank, which=("v",))["v"].cuda()
     steps_qk = [synth.schedule_qk_device(fields, st, seed=args.seed + rank, n_steps=wl.n_steps)
                 for st in range(wl.n_steps)]
     del fields
     stream = torch.cuda.current_stream()
-
-    def run_loop(count_flops=False):
-        flops = 0.0
+    def run_loop(count_flops=False, events=None):
+        flops = []
         for st in range(wl.n_steps):
-            refresh = schedule.is_refresh(st, wl.refresh)
-            if refresh:
-                layer.set_budget(k=schedule.keep_budget(st, s.nb, wl.n_steps, wl.refresh))
-            layer.forward(steps_qk[st]["q"], steps_qk[st]["k"], v, refresh_mask=refresh)
+            if refresh[st]:
+                layer.set_budget(k=ks[st])
+            layer.prepare(steps_qk[st]["q"], steps_qk[st]["k"], v, refresh_mask=refresh[st])
+            if events is not None:
+                events[st][0].record(stream)
+            layer.attend()
+            if events is not None:
+                events[st][1].record(stream)
             if count_flops:
                 torch.cuda.synchronize()
-                flops += 4.0 * wl.D * layer.kept_pairs()
+                flops.append(4.0 * wl.D * layer.kept_pairs())
         return flops
 
-    flops_loop = run_loop(count_flops=True)       # also the first warm-up pass
+    flops_steps = run_loop(count_flops=True)       # also the first warm-up pass
+    flops_loop = sum(flops_steps)
     for _ in range(max(0, args.warmup - 1)):
         run_loop()
     torch.cuda.synchronize()
     assert dfsattn.dfs_get_error_flags(clear=True) == 0
     reps = max(1, min(args.steps, 5))
+    ev_attn = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(wl.n_steps)] for _ in range(reps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
@@ -527,100 +542,188 @@ def run_schedule(args, wl, rank, world, local):
     barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(reps):
-        run_loop()
+    for r in range(reps):
+        run_loop(events=ev_attn[r])
     e1.record(stream)
     torch.cuda.synchronize()
+    attn_ms = [[a.elapsed_time(b) for a, b in evs] for evs in ev_attn]
     barrier(world)
     clk = clocks.stop() if clocks else None
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = ms / (reps * wl.n_steps)
     flops_all = sum_over_ranks(flops_loop * reps, world)
+    attn_total_ms = sum(sum(x) for x in attn_ms)
+
+    # end to end through the public API: every step copies its Q, K, V in from
+    # pinned host memory and its output back (DfsLayer.run_host_steps with the
+    # loop's refresh flags and budgets). Host inputs: the first few steps' Q/K
+    # (the kept counts, hence the work, depend only on the budgets).
+    n_host = 3
+    hv = v.cpu().pin_memory()
+    host_sets = [(steps_qk[i]["q"].cpu().pin_memory(), steps_qk[i]["k"].cpu().pin_memory(), hv) for i in range(n_host)]
+    hos = [torch.empty_like(hv).pin_memory() for _ in range(2)]
+    e2e_inputs = [host_sets[i % n_host] for i in range(wl.n_steps)]
+    e2e_outs = [hos[i & 1] for i in range(wl.n_steps)]
+    set_k = lambda i: layer.set_budget(k=ks[i]) if refresh[i] else None
+    layer.run_host_steps(e2e_inputs, e2e_outs, refresh_mask=refresh, before_step=set_k)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    layer.run_host_steps(e2e_inputs, e2e_outs, refresh_mask=refresh, before_step=set_k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / wl.n_steps
+    assert dfsattn.dfs_get_error_flags(clear=True) == 0
     if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops_loop * reps / (attn_total_ms * 1e-3) / 1e12
         line = {"metric": METRIC, "value": round(flops_all / (ms * 1e-3) / 1e12, 3),
                 "unit": "TFLOP/s (kept-block, amortised over the 50-step loop)", "n_gpus": world,
                 "steps": reps * wl.n_steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+                "attn_ms_per_call": round(attn_total_ms / (reps * wl.n_steps), 4),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded fields; per-step noise drawn on the device)",
-                "config": {"workload": (f"{wl.name}: B={wl.B} nh={wl.nh} D={wl.D} grid {wl.T}x{wl.H}x{wl.W} "
-                                        f"(N={wl.N}), {wl.n_steps} steps, top-k 103 -> 32 of {s.nb}, "
-                                        f"mask refresh every {wl.refresh} steps, attention every step"),
-                           "parallelism": f"replicas x{world}"},
-                "gpu_launches": None, "clocks": clk}
+                "config": {"workload": schedule_config(wl), "kept_pairs_per_loop": int(flops_loop / (4.0 * wl.D)),
+                           "l2": "inputs larger than L2 (3 x %.1f MB of Q/K/V per step)" % (wl.N * wl.nh * wl.D * 2 / 1e6),
+                           "parallelism": f"replicas x{world} (independent layer per GPU)", "launch": "eager launches"},
+                "roofline": {"kernel": "attn_fwd_kernel (inverse reorder fused into the epilogue), over the 50 steps",
+                             "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                             "frac": round(achieved / peak, 4), "peak_source": f"{src} bf16 burst",
+                             "traffic": None},
+                "e2e": {"value": round(sum_over_ranks(flops_loop, world) / (e2e_ms * wl.n_steps * 1e-3) / 1e12, 3),
+                        "unit": "TFLOP/s (kept-block, amortised over the 50-step loop)",
+                        "ms_per_step": round(e2e_ms, 3),
+                        "h2d_bytes_per_step": int(3 * hv.numel() * hv.element_size()),
+                        "d2h_bytes_per_step": int(hv.numel() * hv.element_size()),
+                        "api": "DfsLayer.run_host_steps (per-step refresh flags and budgets; copies overlap the kernels)"},
+                # per step: 3 gathers (or the fused gather + pooling, score and select) and the attention
+                "gpu_launches": 4 * wl.n_steps * reps, "clocks": clk}
+        if not args.no_cpu_baseline and world == 1:
+            qkv = {"q": steps_qk[0]["q"].cpu(), "k": steps_qk[0]["k"].cpu(), "v": hv}
+            wl_sel = synth.Workload(**{**wl.__dict__, "mode": "topk"})
+            line["cpu_baseline"] = cpu_baseline(wl_sel, qkv, ks[0], 0, budget_s=args.cpu_seconds,
+                                                schedule_ks=(ks, refresh))
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
 
 
-def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, steps=1):
-    """Times the oracle on the host over a bounded sample of the workload.
+def oracle_masks(wl, qkv, k, cap, heads, permt):
+    """Curve-ordered fp64 heads and the oracle's kept lists for them."""
+    from oracle import lvsa, radial, scoring, selection
+    per_head = []
+    m = None
+    for h in heads:
+        qp, kp, vp = (qkv[n][0, permt, h, :].double().numpy()[None, None] for n in ("q", "k", "v"))
+        if wl.mode == "lvsa":
+            m = lvsa.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step) if m is None else m
+            idx, cnt = selection.mask_to_lists(m[None, None])
+        elif wl.mode == "radial":
+            m = (radial.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.radial_w0,
+                                   radial.w_far_of(wl.radial_lambda, wl.radial_w0)) if m is None else m)
+            idx, cnt = selection.mask_to_lists(m[None, None])
+        elif wl.mode == "global":
+            sc = scoring.block_scores(qp, kp, wl.blk, wl.sb)
+            idx, cnt = selection.select_global(sc, k)
+        else:
+            sc = scoring.block_scores(qp, kp, wl.blk, wl.sb)
+            idx, cnt = selection.select(sc, "threshold" if wl.mode == "threshold" else "topk", k=k, tau=wl.tau,
+                                        cap=cap, kcap=wl.nb)
+        per_head.append((qp, kp, vp, idx, cnt))
+    return per_head
 
-    The sample: the curve index, scoring and selection over the whole layer,
-    then attention on as many randomly chosen query blocks as fit the time
-    budget; the time per query block is scaled to the whole layer.
-    Returns the oracle's whole-step throughput in the same unit."""
+
+def cpu_baseline(wl, qkv, k, cap, budget_s=20.0, schedule_ks=None):
+    """Times the oracle on the host cores over a bounded sample of the
+    workload and scales it to a whole step: a sampled estimate, not a run of
+    the whole layer.
+
+    Sample: the curve index; scoring and selection head by head (numpy's own
+    threads) until about 40 % of the budget is spent, the remaining heads
+    scaled from their mean; then fp64 attention of random query blocks of the
+    scored heads (at most 4), dealt over all host cores by a pool of spawned
+    processes (oracle.parallel), batch after batch until the budget is
+    spent; the wall time per query block is scaled to every row of the layer.
+    ``schedule_ks`` (one k per denoising step, refresh flags) scales the
+    sample, taken at the first step's budget, to the whole loop: masks at the
+    refresh steps, attention every step in proportion to its k.
+    Returns the estimated whole-step throughput in the bench's unit."""
     import torch
-    from oracle import attention, hilbert, lvsa, radial, scoring, selection
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    from oracle import attention, hilbert, parallel
+    wall0 = time.perf_counter()
     t0 = time.perf_counter()
     perm, _ = hilbert.make_perm(wl.order, wl.T, wl.H, wl.W)
     permt = torch.from_numpy(perm.astype(np.int64))
     t_perm = time.perf_counter() - t0
     rng = np.random.default_rng(0)
-    t_mask = 0.0
-    t_attn = 0.0
-    n_rows = 0
-    kept = 0
     per_head = []
+    t_mask = 0.0
+    t0 = time.perf_counter()
     for h in range(wl.nh):
         t1 = time.perf_counter()
-        qp, kp, vp = (qkv[n][0, permt, h, :].double().numpy()[None, None] for n in ("q", "k", "v"))
-        if wl.mode == "lvsa":
-            m = lvsa.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step) if h == 0 else m
-            idx, cnt = selection.mask_to_lists(m[None, None])
-        elif wl.mode == "radial":
-            m = radial.block_mask(wl.T, wl.H * wl.W, wl.blk, wl.radial_w0,
-                                  radial.w_far_of(wl.radial_lambda, wl.radial_w0)) if h == 0 else m
-            idx, cnt = selection.mask_to_lists(m[None, None])
-        else:
-            sc = scoring.block_scores(qp, kp, wl.blk, wl.sb)
-            idx, cnt = selection.select(sc, wl.mode, k=k, tau=wl.tau, cap=cap)
+        per_head += oracle_masks(wl, qkv, k, cap, [h], permt)
         t_mask += time.perf_counter() - t1
-        per_head.append((qp, kp, vp, idx, cnt))
-        if time.perf_counter() - t0 > budget_s * 0.6 and h < wl.nh - 1:
-            # scoring of the remaining heads is estimated from the mean so far
-            t_mask = t_mask / (h + 1) * wl.nh
+        if time.perf_counter() - t0 > budget_s * 0.4 and h < wl.nh - 1:
             break
     heads_done = len(per_head)
-    allowed = None
+    t_mask = t_mask / heads_done * wl.nh * wl.B
+    att_heads = per_head[:4]
+    stack = lambda i: np.concatenate([ph[i] for ph in att_heads], axis=1)
+    frame = None
     if wl.frame_exact:
-        fa = lvsa.frame_allowed(wl.T, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step)
-        P = wl.H * wl.W
-        allowed = lambda qs, ks: fa[np.asarray(qs)[:, None] // P, np.asarray(ks)[None, :] // P]
-    deadline = time.perf_counter() + max(1.0, budget_s - (time.perf_counter() - t0))
+        from oracle import lvsa
+        frame = (lvsa.frame_allowed(wl.T, wl.lvsa_T_per, wl.lvsa_C, wl.lvsa_step), wl.H * wl.W)
     rows_total = wl.nb * wl.nh * wl.B
-    while time.perf_counter() < deadline:
-        h = int(rng.integers(0, heads_done))
-        I = int(rng.integers(0, wl.nb))
-        qp, kp, vp, idx, cnt = per_head[h]
-        t1 = time.perf_counter()
-        attention.block_sparse_attention(qp, kp, vp, idx, cnt, wl.blk, rows=[(0, 0, I)], allowed=allowed)
-        t_attn += time.perf_counter() - t1
-        n_rows += 1
-        rows_q = min(wl.blk, wl.N - I * wl.blk)
-        c = int(cnt[0, 0, I])
-        js = idx[0, 0, I, :c]
-        kept += rows_q * int(sum(min(wl.blk, wl.N - j * wl.blk) for j in js))
-    t_attn_full = t_attn / max(1, n_rows) * rows_total
-    t_step = t_perm + t_mask + t_attn_full
-    kept_full = kept / max(1, n_rows) * rows_total
-    flops = 4.0 * wl.D * kept_full
-    return {"value": round(flops / t_step / 1e12, 6), "unit": "TFLOP/s (kept-block, whole step)",
-            "cores": threads, "kind": "oracle",
-            "ms_per_step": round(t_step * 1e3, 1),
-            "sample": (f"curve index; scoring+selection on {heads_done}/{wl.nh} heads (rest scaled); "
-                       f"fp64 attention on {n_rows} random query blocks of {rows_total} (scaled)")}
+    n_rows = kept = 0
+    t_attn = 0.0
+    with parallel.RowPool(stack(0), stack(1), stack(2), stack(3), stack(4), wl.blk, frame=frame) as pool:
+        cores = pool.workers
+        # start every worker process (spawned on demand, one per pending task): not timed
+        pool.run([(0, 0, I % wl.nb) for I in range(cores)], blocks_per_task=1)
+        deadline = time.perf_counter() + max(2.0, budget_s - (time.perf_counter() - t0))
+        batch = 4 * cores
+        while True:
+            rows = sorted({(0, int(rng.integers(0, len(att_heads))), int(rng.integers(0, wl.nb)))
+                           for _ in range(batch)})
+            t1 = time.perf_counter()
+            pool.run(rows)
+            dt = time.perf_counter() - t1
+            t_attn += dt
+            n_rows += len(rows)
+            for (_, h, I) in rows:
+                idx, cnt = att_heads[h][3], att_heads[h][4]
+                rows_q = min(wl.blk, wl.N - I * wl.blk)
+                js = idx[0, 0, I, :int(cnt[0, 0, I])]
+                kept += rows_q * int(sum(min(wl.blk, wl.N - j * wl.blk) for j in js))
+            left = deadline - time.perf_counter()
+            if left < 1.5 * dt:
+                break
+            batch = max(4 * cores, min(32 * cores, int(batch * left / max(dt, 1e-3) / 2)))
+    t_attn_full = t_attn / n_rows * rows_total
+    kept_full = kept / n_rows * rows_total
+    # the curve index is built once per grid shape (the GPU path builds it
+    # before timing too); it is reported, not counted in a step
+    if schedule_ks is None:
+        t_step = t_mask + t_attn_full
+        flops = 4.0 * wl.D * kept_full
+        unit = "TFLOP/s (kept-block, whole step)"
+        what = "one step"
+    else:
+        ks, refresh = schedule_ks
+        k0 = ks[0]
+        t_step = (sum(t_mask for r in refresh if r) + sum(t_attn_full * kk / k0 for kk in ks)) / len(ks)
+        flops = sum(4.0 * wl.D * kept_full * kk / k0 for kk in ks) / len(ks)
+        unit = "TFLOP/s (kept-block, amortised over the 50-step loop)"
+        what = f"the {len(ks)}-step loop (sample at k = {k0}, attention scaled by k, masks at {sum(refresh)} refreshes)"
+    return {"value": round(flops / t_step / 1e12, 6), "unit": unit, "cores": cores, "kind": "oracle",
+            "sampled": True, "ms_per_step": round(t_step * 1e3, 1),
+            "wall_s": round(time.perf_counter() - wall0, 2),
+            "curve_index_s": round(t_perm, 2),
+            "sample": (f"estimate of {what} (the curve index, built once per grid, not counted): gather, scoring+selection on {heads_done}/{wl.nh} heads "
+                       f"(numpy threads; rest scaled); fp64 attention of {n_rows} randomly drawn query blocks (the layer has "
+                       f"{rows_total}) over {cores} worker processes, wall time scaled to every row")}
 
 
 def run_reference(args):
@@ -630,25 +733,44 @@ def run_reference(args):
         return
     import synth
     wl = synth.WORKLOADS[args.workload]
-    qkv = synth.workload_inputs(wl, seed=args.seed)
-    k = wl.ratio_count(wl.keep_num) if wl.mode == "topk" else 0
-    cap = wl.ratio_count(wl.cap_num) if wl.mode == "threshold" else 0
-    # seconds of oracle work per timed step (warm-up steps a quarter of it):
-    # 2 to 20 s so that the whole run stays within a few minutes, and never
-    # more than --cpu-seconds
+    sched = None
+    if wl.mode == "schedule":
+        from block_sparse_attention_36_b200 import schedule as hs
+        ks = [hs.keep_budget(st, wl.nb, wl.n_steps, wl.refresh) for st in range(wl.n_steps)]
+        sched = (ks, [hs.is_refresh(st, wl.refresh) for st in range(wl.n_steps)])
+        qkv = dict(synth.schedule_qk(wl.T, wl.H, wl.W, wl.nh, wl.D, 0, seed=args.seed))
+        qkv["v"] = synth.field_qkv(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=args.seed, which=("v",))["v"]
+        wl_sel = synth.Workload(**{**wl.__dict__, "mode": "topk"})
+        k, cap = ks[0], 0
+    else:
+        qkv = synth.workload_inputs(wl, seed=args.seed)
+        wl_sel = wl
+        k = (wl.ratio_count(wl.keep_num) if wl.mode == "topk" else
+             wl.pair_count(wl.keep_num) if wl.mode == "global" else 0)
+        cap = wl.ratio_count(wl.cap_num) if wl.mode == "threshold" else 0
+    # seconds of oracle work per timed estimate (warm-up estimates a quarter
+    # of it): 2 to 20 s so that the whole run stays within a few minutes, and
+    # never more than --cpu-seconds
     budget = max(min(2.0, args.cpu_seconds), min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_baseline(wl, qkv, k, cap, budget_s=budget / 4)
-    vals = [cpu_baseline(wl, qkv, k, cap, budget_s=budget) for _ in range(args.steps)]
+        cpu_baseline(wl_sel, qkv, k, cap, budget_s=budget / 4, schedule_ks=sched)
+    t0 = time.perf_counter()
+    vals = [cpu_baseline(wl_sel, qkv, k, cap, budget_s=budget, schedule_ks=sched) for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
     ms = statistics.mean(v["ms_per_step"] for v in vals)
     val = statistics.mean(v["value"] for v in vals)
     unit = vals[0]["unit"]
+    cfg = schedule_config(wl) if sched else workload_config(wl, k, cap)
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_config(wl, k, cap), "parallelism": "host cores, rank 0 only"},
+            "sampled": True,
+            "sampling": (f"each of the {args.steps} timed steps is one sampled estimate of a whole step "
+                         f"(ms_per_step is the estimated whole-step time); the {args.steps} estimates took "
+                         f"{wall:.1f} s of wall time"),
+            "config": {"workload": cfg, "parallelism": "host cores, rank 0 only"},
             "cpu_baseline": {"value": round(val, 6), "unit": unit, "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": vals[0]["sample"]},
+                             "sampled": True, "sample": vals[0]["sample"]},
             "e2e": {"value": round(val, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -658,7 +780,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="wan_1p3b_layer")
+    ap.add_argument("--workload", default="hunyuan_layer")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)

@@ -150,18 +150,24 @@ class DfsLayer:
         self.attend(stream, out)
         return self.out if out is None else out
 
-    def run_host_steps(self, host_inputs, host_outputs, refresh_mask=True):
+    def run_host_steps(self, host_inputs, host_outputs, refresh_mask=True, before_step=None):
         """Runs one step per (q, k, v) of ``host_inputs`` (pinned host bf16
         [B, N, nh, D]) and copies each result into the matching pinned host
         tensor of ``host_outputs``. Steps are pipelined over three streams:
         the host-to-device copy of step i+1 and the device-to-host copy of
         step i-1 overlap the kernels of step i (two device input sets and two
-        output buffers, ordered by events). Enqueues the work after the
-        current stream's pending work and makes the current stream wait for
-        all of it; returns without synchronising."""
+        output buffers, ordered by events). ``refresh_mask`` is one flag for
+        every step or a sequence with one flag per step (a denoising loop
+        with a cached mask); ``before_step(i)``, if given, is called before
+        step i is enqueued (e.g. to set that step's budget). Enqueues the
+        work after the current stream's pending work and makes the current
+        stream wait for all of it; returns without synchronising."""
         n = len(host_inputs)
         if len(host_outputs) != n:
             raise ValueError("one host output per step")
+        refresh = [bool(refresh_mask)] * n if isinstance(refresh_mask, bool) else [bool(r) for r in refresh_mask]
+        if len(refresh) != n:
+            raise ValueError("one refresh flag per step")
         s = self.shape
         dev = self.qp.device
         if self._pipe is None:
@@ -191,7 +197,9 @@ class DfsLayer:
             s_cmp.wait_event(in_ready)
             if out_done[b] is not None:
                 s_cmp.wait_event(out_done[b])          # step i-2's result has left this buffer
-            self.forward(inp[0], inp[1], inp[2], refresh_mask, stream=s_cmp, out=dout)
+            if before_step is not None:
+                before_step(i)
+            self.forward(inp[0], inp[1], inp[2], refresh[i], stream=s_cmp, out=dout)
             cmp_done[b] = torch.cuda.Event()
             cmp_done[b].record(s_cmp)
             s_out.wait_event(cmp_done[b])

@@ -175,3 +175,32 @@ def test_backward_empty_row_contributes_nothing():
     assert (dk[0, 0, 8:] == 0).all() and (dv[0, 0, 8:] == 0).all()
     ref_q, ref_k, ref_v = attention.block_sparse_attention_bwd(q, k, v, do, idx, cnt, 8, rows=[(0, 0, 1)])
     assert np.array_equal(dk, ref_k) and np.array_equal(dv, ref_v)
+
+
+def test_parallel_rows_equal_the_serial_call():
+    """oracle.parallel only deals query blocks out to worker processes: every
+    row it returns is bitwise the serial oracle's, with and without the
+    frame rule."""
+    from oracle import lvsa, parallel
+    rng = np.random.default_rng(5)
+    B, nh, N, D, blk = 1, 2, 700, 16, 64
+    nb = -(-N // blk)
+    q, k, v = (rng.standard_normal((B, nh, N, D)) for _ in range(3))
+    idx = np.full((B, nh, nb, 5), -1, np.int32)
+    cnt = rng.integers(0, 6, size=(B, nh, nb)).astype(np.int32)
+    for h in range(nh):
+        for I in range(nb):
+            idx[0, h, I, :cnt[0, h, I]] = np.sort(rng.choice(nb, cnt[0, h, I], replace=False))
+    rows = [(0, h, I) for h in range(nh) for I in range(nb)]
+    P = 100
+    fa = lvsa.frame_allowed(7, 3, 4, 1)
+    for frame in (None, (fa, P)):
+        allowed = None if frame is None else (lambda qs, ks: fa[np.asarray(qs)[:, None] // P,
+                                                               np.asarray(ks)[None, :] // P])
+        ref_o, ref_l = attention.block_sparse_attention(q, k, v, idx, cnt, blk, allowed=allowed)
+        got = parallel.block_sparse_attention_rows(q, k, v, idx, cnt, blk, rows, frame=frame, workers=3)
+        assert sorted(got) == sorted(rows)
+        for (b, h, I), (o, l) in got.items():
+            lo, hi = I * blk, min(N, I * blk + blk)
+            assert np.array_equal(o, ref_o[b, h, lo:hi], equal_nan=True)
+            assert np.array_equal(l, ref_l[b, h, lo:hi])
