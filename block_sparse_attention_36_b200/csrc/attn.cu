@@ -54,6 +54,12 @@
 #ifndef DFS_ATTN_EXP2_EMU
 #define DFS_ATTN_EXP2_EMU 0
 #endif
+// 1: with 128-key blocks, S(j+1) is formed in two 64-key halves, the upper
+// one (TMEM columns that P(j) does not occupy) as soon as the softmax has
+// read S(j), the lower one after P.V(j) has read P(j).
+#ifndef DFS_ATTN_EARLY_S
+#define DFS_ATTN_EARLY_S 0
+#endif
 
 namespace {
 
@@ -85,8 +91,9 @@ struct Cfg {
 struct __align__(8) Barriers {
   uint64_t q_full[2];
   uint64_t kv_full[kRing], kv_empty[kRing];
-  uint64_t s_full[2], p_half[2], p_full[2], o_final[2];
+  uint64_t s_full[2], s_read[2], p_half[2], p_full[2], o_final[2];
   uint64_t mma_done;
+  uint64_t stall;          // nothing ever arrives here (the abort-path test)
   uint32_t tmem_base;
   int abort_flag;
   int n_kv[2];
@@ -102,6 +109,21 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t d
     const uint64_t oa = (uint64_t)(((kk >> 2) * (kQRows * 128) + (kk & 3) * 32) >> 4);
     const uint64_t ob = (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
     mma_ss_warp(d_tmem, dq + oa, dk + ob, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// One 64-key half of S = Q K^T (keys 64 h .. 64 h + 63 of the tile, into
+// TMEM columns d_tmem + 0 .. 63): K rows 64 h .. start 64 h * 128 bytes into
+// each 128-byte-wide slab of the tile.
+template <int D, int BLK>
+__device__ __forceinline__ void issue_s_half(uint32_t d_tmem, uint64_t dq, uint64_t dk, int h) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kQRows, 64, 0);
+  const uint64_t row0 = (uint64_t)((h * 64 * 128) >> 4);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t oa = (uint64_t)(((kk >> 2) * (kQRows * 128) + (kk & 3) * 32) >> 4);
+    const uint64_t ob = (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
+    mma_ss_warp(d_tmem, dq + oa, dk + ob + row0, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -136,6 +158,9 @@ struct FrameMask {
 // the epilogue merges the two partial softmax states. The host sets
 // split_from so that the last, partial wave of two-row CTAs becomes twice
 // as many half-length CTAs (tail_split) or leaves it at the CTA count.
+// stall_cycles > 0 (tests only): the MMA-issuing warp first waits that many
+// SM cycles on the barrier `stall`, which nothing arrives at, so the launch
+// runs the abort path of a bounded wait that gives up.
 struct OutMap {
   const int32_t* perm;
   int nh;
@@ -143,6 +168,7 @@ struct OutMap {
   long long rows;
   int tail_split;
   long long split_from;
+  long long stall_cycles;
 };
 
 constexpr int kFrameRows = 3;
@@ -192,6 +218,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->q_full[x], 1);
       mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->s_read[x], 4);
       mbar_init(&bars->p_half[x], 4);
       mbar_init(&bars->p_full[x], 4);
       mbar_init(&bars->o_final[x], 1);
@@ -201,6 +228,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&bars->kv_empty[s], 1);
     }
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->stall, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
     // Q of each existing slot depends only on its block index: start both
@@ -294,7 +322,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         prefetch_tensor_map(&tm_v);
       }
       // Same step order as the MMA issuer: step -1 loads K_A(0), K_B(0); step
-      // j loads, per slot, V(j) and then K(j+1).
+      // j loads, per slot, V(j) and then K(j+1) (with the early S halves:
+      // K(j+1) first, its upper half is read before P.V(j)).
+      constexpr bool kEarly = DFS_ATTN_EARLY_S && BLK == 128;
       int t = 0;  // ring tiles loaded so far
       bool ok = true;
       for (int step = -1; step < jmax && ok; ++step) {
@@ -303,7 +333,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int nx = n[x];
           if (step >= nx) continue;
 #pragma unroll 1
-          for (int kind = 0; kind < 2; ++kind) {      // 0: V(step), 1: K(step + 1)
+          for (int kk2 = 0; kk2 < 2; ++kk2) {
+            const int kind = kEarly ? 1 - kk2 : kk2;  // 0: V(step), 1: K(step + 1)
             const int jj = kind == 0 ? step : step + 1;
             if (jj < 0 || jj >= nx) continue;
             const int st = t % kRing;
@@ -341,6 +372,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t dk = desc_sw128(smem_addr(smem + C::kRingOff), 16, 1024);
       const uint64_t dv = desc_sw128(smem_addr(smem + C::kRingOff), BLK * 128, 1024);
       bool ok = true;
+      if (om.stall_cycles > 0) ok = mbar_wait_bounded(&bars->stall, 0, abort_flag, om.stall_cycles);
       for (int x = 0; x < 2 && ok; ++x)
         if (n[x] > 0) ok = mbar_wait_bounded(&bars->q_full[x], 0, abort_flag, kWaitLimit);
       // Step -1 issues S_A(0), S_B(0); step j issues, per slot, PV(j) and
@@ -351,6 +383,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int x = 0; x < 2; ++x) {
           const int nx = n[x];
           if (step >= nx) continue;
+          if (DFS_ATTN_EARLY_S && BLK == 128 && step >= 0) {
+            // ring order: K(step + 1) [stage tk], then V(step) [stage tv]
+            const bool more = step + 1 < nx;
+            const int tk = t, tv = more ? t + 1 : t;
+            const uint64_t dqx = dq + (uint64_t)((x * C::kQBytes) >> 4);
+            const uint64_t dks = dk + (uint64_t)(((tk % kRing) * C::kTileBytes) >> 4);
+            const uint32_t s_tm = tmem + C::s_col(x);
+            if (more) {
+              // keys 64-127 of S(step + 1) go to columns P(step) leaves free,
+              // once the softmax has read S(step)
+              if (!mbar_wait_bounded(&bars->s_read[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              if (!mbar_wait_bounded(&bars->kv_full[tk % kRing], (uint32_t)((tk / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+              tc_fence_after();
+              issue_s_half<D, BLK>(s_tm + 64, dqx, dks, 1);
+            }
+            const uint64_t dvs = dv + (uint64_t)(((tv % kRing) * C::kTileBytes) >> 4);
+            if (!mbar_wait_bounded(&bars->p_half[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+            tc_fence_after();
+            if (!mbar_wait_bounded(&bars->kv_full[tv % kRing], (uint32_t)((tv / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+            issue_pv<D, BLK, 0, BLK / 32>(tmem + C::o_col(x), s_tm, dvs, step > 0);
+            if (!mbar_wait_bounded(&bars->p_full[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv<D, BLK, BLK / 32, BLK / 16>(tmem + C::o_col(x), s_tm, dvs, true);
+            mma_commit_warp(&bars->kv_empty[tv % kRing]);
+            if (more) {
+              issue_s_half<D, BLK>(s_tm, dqx, dks, 0);   // keys 0-63, over P(step) once P.V(step) has read it
+              mma_commit_warp(&bars->s_full[x]);
+              mma_commit_warp(&bars->kv_empty[tk % kRing]);
+            } else {
+              mma_commit_warp(&bars->o_final[x]);
+            }
+            t += more ? 2 : 1;
+            continue;
+          }
           if (step >= 0) {
             // P_X was written by other threads with tcgen05.st: order this
             // thread's MMAs after their arrival. (TMA-filled tiles need no
@@ -424,6 +490,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[e]);
       }
       tmem_wait_ld();
+      if (DFS_ATTN_EARLY_S && BLK == 128) {
+        // S(j) is in registers: its columns may take the next S
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_read[x]);
+      }
       if (list[j] == nb - 1 && rem < BLK) {
 #pragma unroll
         for (int e = 0; e < BLK; ++e)
@@ -742,7 +814,7 @@ extern "C" int dfs_sparse_attn_fwd(const dfs_shape* shape, const void* qp, const
   if (st != DFS_OK) return st;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
   return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream,
-                              FrameMask{1, 1, 1, 0, 1, 0}, OutMap{nullptr, 1, nullptr, d.BH * d.nb, 1, 0});
+                              FrameMask{1, 1, 1, 0, 1, 0}, OutMap{nullptr, 1, nullptr, d.BH * d.nb, 1, 0, 0});
 }
 
 extern "C" int dfs_sparse_attn_fwd_ex(const dfs_shape* shape, const void* qp, const void* kp, const void* vp,
@@ -752,11 +824,12 @@ extern "C" int dfs_sparse_attn_fwd_ex(const dfs_shape* shape, const void* qp, co
   const int st = check_attn_args(shape, qp, kp, vp, kv_idx, kv_cnt, kcap, o, lse, &d);
   if (st != DFS_OK) return st;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d.D);
-  OutMap om{nullptr, d.nh, nullptr, d.BH * d.nb, 1, 0};
+  OutMap om{nullptr, d.nh, nullptr, d.BH * d.nb, 1, 0, 0};
   if (opts) {
     om.perm = opts->perm;
     om.order = opts->order;
     om.tail_split = opts->no_tail_split ? 0 : 1;
+    om.stall_cycles = (long long)opts->test_stall_cycles;
   }
   return dispatch_attn<false>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse, (cudaStream_t)stream,
                               FrameMask{1, 1, 1, 0, 1, 0}, om);
@@ -780,42 +853,100 @@ extern "C" int dfs_sparse_attn_lvsa_fwd(const dfs_shape* shape, const void* qp, 
   fm.C = lvsa->lvsa_C;
   fm.nG = (fm.s0 < d.T) ? (d.T - 1 - fm.s0) / fm.T_per + 1 : 0;
   return dispatch_attn<true>(d, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, op, lse, (cudaStream_t)stream, fm,
-                             OutMap{nullptr, 1, nullptr, d.BH * d.nb, 1, 0});
+                             OutMap{nullptr, 1, nullptr, d.BH * d.nb, 1, 0, 0});
 }
 
 namespace {
 
-// Counting sort of the query rows by kept count, descending, in one CTA:
-// shared-memory histogram, a scan from the largest count down, and a
-// scatter through per-count cursors (warp-aggregated, so rows of equal
-// count keep their order inside a warp's 32-row chunk).
-__global__ void __launch_bounds__(1024)
-attn_order_kernel(const int32_t* __restrict__ kv_cnt, long long rows, int kmax, int32_t* __restrict__ order) {
-  extern __shared__ int cursor[];   // kmax + 1 counters
-  const int tid = threadIdx.x, lane = tid & 31;
-  for (int c = tid; c <= kmax; c += blockDim.x) cursor[c] = 0;
+// Stable counting sort of the query rows of one head (one CTA per head) by
+// kept count, descending: rows of equal count stay in ascending order, so
+// the order (and every result computed in it) is the same on every run, and
+// the heads stay in order, so the CTAs running at any time read the keys and
+// values of about two heads (they stay in L2).
+//   1. warp w < S takes the contiguous segment w of the head's rows and
+//      counts its keys into its own histogram hist[w][key] (only warp w
+//      writes it);
+//   2. the key totals are scanned from the largest key down, and each
+//      histogram entry becomes the first output slot of that warp's rows
+//      with that key: base(key) + rows of that key in segments before w;
+//   3. each warp walks its segment in order, 32 rows at a time; the lanes
+//      with equal keys (__match_any_sync) take consecutive slots in lane
+//      order and the group's leader advances hist[w][key].
+// S = the number of segments whose histograms fit the shared memory.
+constexpr int kOrderThreads = 1024;
+constexpr size_t kOrderSmemMax = 200 * 1024;
+
+__host__ __device__ inline int order_segments(int kmax) {
+  const long long per = (long long)(kmax + 1) * (long long)sizeof(int);
+  const long long s = (long long)kOrderSmemMax / per - 1;    // one row of the table holds the key bases
+  return (int)(s < 1 ? 1 : (s > kOrderThreads / 32 ? kOrderThreads / 32 : s));
+}
+
+__global__ void __launch_bounds__(kOrderThreads)
+attn_order_kernel(const int32_t* __restrict__ kv_cnt, int nb, int kmax, int nseg, int32_t* __restrict__ order) {
+  extern __shared__ int hist[];              // [nseg + 1][kmax + 1]; the last row: key bases
+  const int K = kmax + 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long row0 = (long long)blockIdx.x * nb;   // this head's rows: row0 .. row0 + nb - 1
+  const int32_t* cnt = kv_cnt + row0;
+  int32_t* out = order + row0;
+  int* base = hist + (size_t)nseg * K;
+  for (int i = tid; i < (nseg + 1) * K; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (long long r = tid; r < rows; r += blockDim.x) atomicAdd(&cursor[max(0, min(kv_cnt[r], kmax))], 1);
+  const int seg = (nb + nseg - 1) / nseg;
+  const int lo = warp * seg, hi = min(lo + seg, nb);
+  int* mine = hist + (size_t)warp * K;
+  if (warp < nseg) {
+    for (int r0 = lo; r0 < hi; r0 += 32) {
+      const int r = r0 + lane;
+      const bool in = r < hi;
+      const int c = in ? max(0, min(cnt[r], kmax)) : -1 - lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      if (in && lane == __ffs(peers) - 1) mine[c] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < K; c += blockDim.x) {
+    int tot = 0;
+    for (int w = 0; w < nseg; ++w) tot += hist[(size_t)w * K + c];
+    base[c] = tot;
+  }
   __syncthreads();
   if (tid == 0) {
     int run = 0;
     for (int c = kmax; c >= 0; --c) {
-      const int h = cursor[c];
-      cursor[c] = run;
+      const int h = base[c];
+      base[c] = run;
       run += h;
     }
   }
   __syncthreads();
-  for (long long r0 = (long long)(tid >> 5) * 32; r0 < rows; r0 += blockDim.x) {
-    const long long r = r0 + lane;
-    const bool in = r < rows;
-    const int c = in ? max(0, min(kv_cnt[r], kmax)) : -1 - lane;
-    const unsigned peers = __match_any_sync(0xffffffffu, c);
-    const int leader = __ffs(peers) - 1;
-    int base = 0;
-    if (in && lane == leader) base = atomicAdd(&cursor[c], __popc(peers));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (in) order[base + __popc(peers & ((1u << lane) - 1u))] = (int32_t)r;
+  for (int c = tid; c < K; c += blockDim.x) {
+    int run = base[c];
+    for (int w = 0; w < nseg; ++w) {
+      const int h = hist[(size_t)w * K + c];
+      hist[(size_t)w * K + c] = run;
+      run += h;
+    }
+  }
+  __syncthreads();
+  if (warp < nseg) {
+    for (int r0 = lo; r0 < hi; r0 += 32) {
+      const int r = r0 + lane;
+      const bool in = r < hi;
+      const int c = in ? max(0, min(cnt[r], kmax)) : -1 - lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      const int leader = __ffs(peers) - 1;
+      int slot = 0;
+      if (in && lane == leader) {
+        slot = mine[c];
+        mine[c] = slot + __popc(peers);
+      }
+      slot = __shfl_sync(0xffffffffu, slot, leader);
+      if (in) out[slot + __popc(peers & ((1u << lane) - 1u))] = (int32_t)(row0 + r);
+      __syncwarp();
+    }
   }
 }
 
@@ -829,7 +960,13 @@ extern "C" int dfs_attn_order(const dfs_shape* shape, const int32_t* kv_cnt, int
   if (!kv_cnt || !order || kcap < 1) return DFS_ERR_INVALID_ARG;
   const int kmax = min(kcap, d.nb);
   if (d.BH * d.nb >= (1LL << 31)) return DFS_ERR_UNSUPPORTED;
-  attn_order_kernel<<<1, 1024, (size_t)(kmax + 1) * sizeof(int), (cudaStream_t)stream>>>(kv_cnt, d.BH * d.nb, kmax,
-                                                                                          order);
+  const int nseg = order_segments(kmax);
+  const size_t smem = (size_t)(nseg + 1) * (kmax + 1) * sizeof(int);
+  if (smem > 232448) return DFS_ERR_UNSUPPORTED;      // two table rows beyond the shared memory: kmax > 29055
+  if (cudaFuncSetAttribute(attn_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return DFS_ERR_CUDA;
+  if (d.BH > 0x7fffffffLL) return DFS_ERR_UNSUPPORTED;
+  attn_order_kernel<<<(unsigned)d.BH, kOrderThreads, smem, (cudaStream_t)stream>>>(kv_cnt, d.nb, kmax, nseg, order);
   return dfs::launch_status();
 }

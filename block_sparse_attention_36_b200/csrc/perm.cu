@@ -151,16 +151,25 @@ __global__ void hilbert_index_kernel(int T, int H, int W, int order, int ct, int
     n = tiled_cell(i, T, H, W, ct, ch, cw);
     if (n < 0 || n >= N) n = 0;  // unreachable for valid shapes; keeps the write in bounds
   } else {
+    // 3-D: the curve of the whole T x H x W box. 2-D (frame-major): frame
+    // t = i / (H W) in time order, its tokens along the curve of the
+    // 1 x H x W box (the same path in every frame).
+    const bool two_d = order == DFS_ORDER_HILBERT2D;
+    const long long P = (long long)H * W;
+    const int Tb = two_d ? 1 : T;
+    const long long t0 = two_d ? i / P : 0;
+    const long long rank = two_d ? i - t0 * P : i;
     // Major axis: the longest side, ties to W, then H, then T; the other two
     // in the order W, H, T.
-    Axis aw{2, W}, ah{1, H}, at{0, T};
+    Axis aw{2, W}, ah{1, H}, at{0, Tb};
     Box top;
     top.p[0] = top.p[1] = top.p[2] = 0;
-    if (W >= H && W >= T) { top.a = aw; top.b = ah; top.c = at; }
-    else if (H >= T) { top.a = ah; top.b = aw; top.c = at; }
+    if (W >= H && W >= Tb) { top.a = aw; top.b = ah; top.c = at; }
+    else if (H >= Tb) { top.a = ah; top.b = aw; top.c = at; }
     else { top.a = at; top.b = aw; top.c = ah; }
     int cell[3];
-    hilbert_cell(top, i, cell);
+    hilbert_cell(top, rank, cell);
+    cell[0] += (int)t0;
     n = ((long long)cell[0] * H + cell[1]) * W + cell[2];
     if (cell[0] < 0 || cell[0] >= T || cell[1] < 0 || cell[1] >= H || cell[2] < 0 || cell[2] >= W)
       n = 0;  // unreachable for valid shapes; keeps the write in bounds
@@ -296,7 +305,7 @@ gather_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, con
 
 bool valid_order(int order) {
   return order == DFS_ORDER_RASTER || order == DFS_ORDER_HILBERT3D || order == DFS_ORDER_TILE2D ||
-         order == DFS_ORDER_TILE3D;
+         order == DFS_ORDER_TILE3D || order == DFS_ORDER_HILBERT2D;
 }
 
 // Tile extents of the tiled orders (blk tokens per full tile).

@@ -40,8 +40,9 @@ DFS_FLAG_KCAP_OVERFLOW = 4
 
 DFS_ORDER_TILE2D = 2
 DFS_ORDER_TILE3D = 3
+DFS_ORDER_HILBERT2D = 4
 ORDERS = {"raster": DFS_ORDER_RASTER, "hilbert3d": DFS_ORDER_HILBERT3D, "tile2d": DFS_ORDER_TILE2D,
-          "tile3d": DFS_ORDER_TILE3D}
+          "tile3d": DFS_ORDER_TILE3D, "hilbert2d": DFS_ORDER_HILBERT2D}
 MODES = {"topk": DFS_SEL_TOPK, "threshold": DFS_SEL_THRESHOLD, "lvsa": DFS_SEL_LVSA, "global": DFS_SEL_GLOBAL,
          "radial": DFS_SEL_RADIAL}
 
@@ -59,7 +60,8 @@ class _Shape(ctypes.Structure):
 
 
 class _AttnOpts(ctypes.Structure):
-    _fields_ = [("perm", ctypes.c_void_p), ("order", ctypes.c_void_p), ("no_tail_split", ctypes.c_int)]
+    _fields_ = [("perm", ctypes.c_void_p), ("order", ctypes.c_void_p), ("no_tail_split", ctypes.c_int),
+                ("test_stall_cycles", ctypes.c_uint)]
 
 
 class _SelectParams(ctypes.Structure):
@@ -299,14 +301,14 @@ def dfs_sparse_attn_fwd(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o
 
 
 def dfs_sparse_attn_fwd_ex(shape: Shape, qp, kp, vp, kv_idx, kv_cnt, kcap, scale, o, lse=None, perm=None,
-                           order=None, stream=None, tail_split=True):
+                           order=None, stream=None, tail_split=True, test_stall_cycles=0):
     c = "dfs_sparse_attn_fwd_ex"
     _need_attn(c, shape, qp, kp, vp, kv_idx, kv_cnt, kcap, o, lse)
     _need(c, "perm", perm, shape.N, _I32, optional=True)
     _need(c, "order", order, _rows(shape), _I32, optional=True)
     sh = shape.c()
     opts = _AttnOpts(None if perm is None else perm.data_ptr(), None if order is None else order.data_ptr(),
-                     0 if tail_split else 1)
+                     0 if tail_split else 1, int(test_stall_cycles))
     _check("dfs_sparse_attn_fwd_ex", LIB.dfs_sparse_attn_fwd_ex(
         ctypes.byref(sh), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(kv_idx), _ptr(kv_cnt), int(kcap), float(scale),
         ctypes.byref(opts), _ptr(o), _ptr(lse), _stream(stream)))

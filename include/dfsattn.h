@@ -62,7 +62,13 @@ typedef struct {
   int blk, sb;
 } dfs_shape;
 
-enum { DFS_ORDER_RASTER = 0, DFS_ORDER_HILBERT3D = 1, DFS_ORDER_TILE2D = 2, DFS_ORDER_TILE3D = 3 };
+enum {
+  DFS_ORDER_RASTER = 0,
+  DFS_ORDER_HILBERT3D = 1,
+  DFS_ORDER_TILE2D = 2,
+  DFS_ORDER_TILE3D = 3,
+  DFS_ORDER_HILBERT2D = 4
+};
 enum { DFS_SEL_TOPK = 0, DFS_SEL_THRESHOLD = 1, DFS_SEL_LVSA = 2, DFS_SEL_GLOBAL = 3, DFS_SEL_RADIAL = 4 };
 enum { DFS_WS_BLOCK_SCORE = 0, DFS_WS_ATTN_BWD = 1 };
 
@@ -126,7 +132,12 @@ typedef struct {
  * "VMoBA: Mixture of Block Attention for Video Diffusion Models" (abstract,
  * modification 1), read as tile-major orders: tiles of 1 x 8 x (blk/8)
  * tokens (one frame) or 2 x 8 x (blk/16) tokens, in raster order over the
- * tile grid, clipped at its far edges, raster order inside each tile.
+ * tile grid, clipped at its far edges, raster order inside each tile;
+ * DFS_ORDER_HILBERT2D is the 2-D Hilbert order that the DFSAttn ablation
+ * (Results, ablation studies) compares against, read as frame-major: the
+ * frames whole and in time order, each frame's H x W tokens along the
+ * generalised Hilbert curve of the 1 x H x W box (the same path in every
+ * frame; the textbook 2-D Hilbert curve on 2^k x 2^k frames).
  * The index depends only on (T, H, W, order): callers build it once and
  * reuse it with build_index = 0.
  * Then gathers each non-NULL input x in {q, k, v}, bf16 [B, N, nh, D]
@@ -247,6 +258,13 @@ typedef struct {
    * unsplit ones by rounding only. Nonzero: every CTA takes two rows.
    * dfs_sparse_attn_fwd and dfs_sparse_attn_lvsa_fwd use the default.      */
   int no_tail_split;
+  /* test_stall_cycles: testing only, 0 in normal use. Nonzero makes every
+   * CTA's MMA-issuing warp first wait, for at most this many SM cycles, on a
+   * barrier that nothing arrives at: the wait gives up, the CTA raises
+   * DFS_FLAG_WAIT_TIMEOUT, drains the copies and MMAs it started, releases
+   * its tensor memory and writes nothing -- the path any wait takes that
+   * gives up (a GPU fault is never needed to test it).                    */
+  unsigned int test_stall_cycles;
 } dfs_attn_opts;
 
 /* dfs_sparse_attn_fwd_ex -- dfs_sparse_attn_fwd with the options above.
@@ -255,12 +273,17 @@ int dfs_sparse_attn_fwd_ex(const dfs_shape *shape, const void *qp, const void *k
                            const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
                            const dfs_attn_opts *opts, void *o, float *lse, dfs_stream_t stream);
 
-/* dfs_attn_order -- a work order for dfs_attn_opts.order: the query rows
- * sorted by kept count (kv_cnt clamped to [0, min(kcap, nb)]), largest
- * first, so the longest rows start first and the two rows of a CTA have
- * equal work (longest-processing-time first for lists of uneven length,
- * as threshold and global selection make). Rows of equal count keep their
- * order within each 32-row chunk. One CTA, no workspace.                   */
+/* dfs_attn_order -- a work order for dfs_attn_opts.order: within each head
+ * the query rows sorted by kept count (kv_cnt clamped to [0, min(kcap,
+ * nb)]), largest first, and the heads in order. The longest rows of a head
+ * start first and the two rows of a CTA have equal work (longest-processing-
+ * time first for lists of uneven length, as threshold and global selection
+ * make), while the CTAs running at any time share the keys and values of
+ * about two heads, which stay in L2. The sort is stable: rows of equal
+ * count stay in ascending row order, so the order -- and with it which rows
+ * a launch's last, split wave takes -- is the same on every run, and so is
+ * every output bit. One CTA per head, no workspace; min(kcap, nb) must not
+ * exceed 29055 (DFS_ERR_UNSUPPORTED).                                       */
 int dfs_attn_order(const dfs_shape *shape, const int32_t *kv_cnt, int kcap, int32_t *order, dfs_stream_t stream);
 
 /* dfs_sparse_attn_lvsa_fwd -- frame-exact LVSA attention (LVSA: Training-Free

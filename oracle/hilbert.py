@@ -158,6 +158,27 @@ def hilbert_perm(T, H, W):
     return perm, inv
 
 
+def hilbert2d_cells(T, H, W):
+    """Frame-major cells with a 2-D Hilbert curve inside every frame.
+
+    Reading of DFSAttn, Results (ablation studies: the 3D Hilbert order is
+    compared with raster scans and with 2-D Hilbert curves; the page does not
+    define the 2-D variant): frames are kept whole and in time order, as a
+    per-frame (spatial-only) curve implies, and every frame's H x W tokens
+    follow the generalised Hilbert curve of that rectangle -- the definition
+    above applied to the 1 x H x W box, which on 2^k x 2^k squares is the
+    textbook 2-D Hilbert curve. Every frame uses the same path."""
+    frame = [(h, w) for (_, h, w) in hilbert_cells(1, H, W)]
+    return [(t, h, w) for t in range(T) for (h, w) in frame]
+
+
+def hilbert2d_perm(T, H, W):
+    perm = raster_index(hilbert2d_cells(T, H, W), H, W).astype(np.int32)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=np.int32)
+    return perm, inv
+
+
 def raster_perm(T, H, W):
     """The identity order (plain row-major flattening used by standard DiTs)."""
     perm = np.arange(T * H * W, dtype=np.int32)
@@ -204,6 +225,8 @@ def tiled_perm(T, H, W, tile):
 def make_perm(order, T, H, W, blk=128):
     if order == "hilbert3d":
         return hilbert_perm(T, H, W)
+    if order == "hilbert2d":
+        return hilbert2d_perm(T, H, W)
     if order == "raster":
         return raster_perm(T, H, W)
     if order in ("tile2d", "tile3d"):

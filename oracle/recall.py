@@ -3,7 +3,7 @@
 DFSAttn: Dynamic Fine-grained Sparse Attention for Efficient Video
 Generation, Methodology (the method is built around a lower bound on
 attention recall) and Results (ablations: the 3D Hilbert order beats raster
-and 2-D orders; smaller sub-blocks score better). The pages give no formula
+scans and 2-D Hilbert curves; smaller sub-blocks score better). The pages give no formula
 for recall; here it is read as the share of each query's dense softmax mass
 that falls on the keys its kept blocks cover, averaged over queries.
 
@@ -68,9 +68,14 @@ def main():
     ap.add_argument("--workload", default="tiny")
     ap.add_argument("--queries", type=int, default=256, help="sampled queries per head")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--input", default="field", choices=["field", "segmented"],
+                    help="smooth fields (the workloads' inputs) or segmented fields with several centroids per block")
     a = ap.parse_args()
     wl = synth.WORKLOADS[a.workload]
-    qkv = synth.field_qkv(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=a.seed, which=("q", "k"))
+    if a.input == "field":
+        qkv = synth.field_qkv(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=a.seed, which=("q", "k"))
+    else:
+        qkv = synth.segmented_qk(wl.T, wl.H, wl.W, wl.nh, wl.D, seed=a.seed)
     q = qkv["q"].double().numpy()
     k = qkv["k"].double().numpy()
     rng = np.random.default_rng(a.seed)
@@ -78,7 +83,7 @@ def main():
     k_keep = selection.ratio_count(wl.keep_num or 15, 100, wl.nb)
     print(f"workload {wl.name}: N={wl.N}, nb={wl.nb}, keep {k_keep}/{wl.nb}, {len(queries)} sampled queries")
     print("| order | sub-block | recall |\n|---|---|---|")
-    for order in ("raster", "tile2d", "tile3d", "hilbert3d"):
+    for order in ("raster", "tile2d", "tile3d", "hilbert2d", "hilbert3d"):
         for sb in (wl.blk, wl.sb):
             r = variant_recall(q, k, wl.T, wl.H, wl.W, wl.blk, sb, order, k_keep, queries)
             print(f"| {order} | {sb}{' (coarse)' if sb == wl.blk else ''} | {r:.4f} |", flush=True)

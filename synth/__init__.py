@@ -169,6 +169,43 @@ def schedule_qk_device(fields, s, seed=0, n_steps=50):
             for n in ("q", "k")}
 
 
+def segmented_qk(T, H, W, nh, D, B=1, seed=0, region_tokens=256, share=0.55, t_scale=4.0):
+    """Q, K with several semantic centroids per block (bf16 CPU [B, N, nh, D]).
+
+    Stand-in for frames of several objects: the grid is cut into Voronoi
+    regions around R = N / region_tokens random sites (time distances
+    weighted by t_scale); region r has a centroid c_r ~ N(0, I) shared by Q
+    and K of the head, so a query attends mostly to keys of its own region,
+    and blocks that straddle a region boundary hold several unrelated
+    centroids. Per token: x = sqrt(share) * g_r * c_r + sqrt(1 - share) * z,
+    z ~ N(0, I) drawn separately for Q and K, g_r ~ U[0.5, 1.5] a per-region
+    strength. Draws: sites and strengths from SeedSequence([seed, b, 7, h]),
+    centroids (R x D) from [seed, b, 8, h], z from [seed, b, tensor_id, h, 99].
+    """
+    N = T * H * W
+    t, h, w = (a.reshape(-1).astype(np.float64) for a in np.meshgrid(np.arange(T), np.arange(H), np.arange(W),
+                                                                      indexing="ij"))
+    out = {n: torch.empty((B, N, nh, D), dtype=torch.bfloat16) for n in ("q", "k")}
+    R = max(2, N // region_tokens)
+    for b in range(B):
+        for hd in range(nh):
+            rs = np.random.default_rng([seed, b, 7, hd])
+            sites = np.stack([rs.uniform(0, T, R), rs.uniform(0, H, R), rs.uniform(0, W, R)], 1)
+            gain = rs.uniform(0.5, 1.5, R)
+            cent = np.random.default_rng([seed, b, 8, hd]).standard_normal((R, D))
+            label = np.empty(N, dtype=np.int64)
+            for lo in range(0, N, 8192):
+                sl = slice(lo, min(N, lo + 8192))
+                d2 = ((t_scale * (t[sl, None] - sites[None, :, 0])) ** 2 + (h[sl, None] - sites[None, :, 1]) ** 2
+                      + (w[sl, None] - sites[None, :, 2]) ** 2)
+                label[sl] = d2.argmin(1)
+            base = math.sqrt(share) * gain[label, None] * cent[label]
+            for name in ("q", "k"):
+                z = np.random.default_rng([seed, b, TENSOR_IDS[name], hd, 99]).standard_normal((N, D))
+                out[name][b, :, hd, :] = _to_bf16(base + math.sqrt(1.0 - share) * z)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # The five workloads (shapes, block sizes and selection settings).
 # ---------------------------------------------------------------------------

@@ -193,9 +193,7 @@ def test_work_order_changes_nothing(lib, B, nh, D, N, kcap):
     lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, b, lb, order=order, tail_split=False)
     torch.cuda.synchronize()
     o = order.cpu().numpy()
-    assert np.array_equal(np.sort(o), np.arange(B * nh * nb))
-    counts = cnt.reshape(-1)[o]
-    assert (np.diff(counts) <= 0).all()
+    assert np.array_equal(o, _per_head_order(cnt, min(kcap, nb)))
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert torch.equal(la, lb)
 
@@ -304,3 +302,113 @@ def test_binding_rejects_wrong_tensors(lib):
         assert e.value.status == lib.DFS_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert bool((op == 7.0).all())
+
+
+def _per_head_order(cnt, kmax):
+    """The rows of each head stably sorted by clamped count, largest first;
+    heads in order (flat row indices)."""
+    c = np.clip(np.asarray(cnt).reshape(-1, np.asarray(cnt).shape[-1]), 0, kmax)
+    nb = c.shape[1]
+    return np.concatenate([bh * nb + np.argsort(-c[bh], kind="stable") for bh in range(c.shape[0])])
+
+
+@pytest.mark.parametrize("nb,kcap,nh", [(929, 186, 24), (2000, 2000, 3), (9000, 9000, 1), (300, 5000, 40)])
+def test_work_order_is_a_stable_sort(lib, nb, kcap, nh):
+    """dfs_attn_order sorts the rows of each head stably by kept count
+    (clamped to min(kcap, nb)), largest first, heads in order: rows of equal
+    count in ascending order -- for small and large count ranges (fewer
+    histogram segments), counts out of range included."""
+    rng = np.random.default_rng(nb + kcap)
+    kmax = min(kcap, nb)
+    cnt = rng.integers(0, kmax + 1, size=(1, nh, nb)).astype(np.int32)
+    cnt.reshape(-1)[::97] = kmax + 3            # clamped to kmax
+    cnt.reshape(-1)[5::101] = -2                # clamped to 0
+    s = lib.Shape(1, nh, 128, 1, 1, nb * 128, 128, 32)
+    order = torch.full((nh * nb,), -1, dtype=torch.int32, device="cuda")
+    lib.dfs_attn_order(s, torch.from_numpy(cnt).cuda(), kcap, order)
+    torch.cuda.synchronize()
+    assert np.array_equal(order.cpu().numpy(), _per_head_order(cnt, kmax))
+
+
+def test_forward_is_reproducible_with_work_order_and_tail_split(lib):
+    """Hunyuan-shaped threshold lists (24 heads, 929 blocks, uneven counts up
+    to the cap of 186, many rows of equal count): two launches in the work
+    order with the default tail split give the same output and LSE bit for
+    bit, and so does a work order built again."""
+    B, nh, D, blk, N, kcap = 1, 24, 128, 128, 118800, 186
+    nb = -(-N // blk)
+    rng = np.random.default_rng(7)
+    cnt = rng.integers(1, kcap + 1, size=(B, nh, nb)).astype(np.int32)
+    idx = np.full((B, nh, nb, kcap), -1, dtype=np.int32)
+    for h in range(nh):
+        for I in range(nb):
+            idx[0, h, I, :cnt[0, h, I]] = np.sort(rng.choice(nb, size=cnt[0, h, I], replace=False))
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, 32)
+    g = torch.Generator(device="cuda").manual_seed(11)
+    qp, kp, vp = (torch.randn((B, nh, N, D), generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    res = []
+    for _ in range(2):
+        order = torch.empty(B * nh * nb, dtype=torch.int32, device="cuda")
+        lib.dfs_attn_order(s, ct, kcap, order)
+        for _ in range(2):
+            o = torch.empty_like(qp)
+            lse = torch.empty((B, nh, N), dtype=torch.float32, device="cuda")
+            lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, o, lse, order=order)
+            res.append((order, o, lse))
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == 0
+    o0 = res[0]
+    for r in res[1:]:
+        assert torch.equal(r[0], o0[0])
+        assert torch.equal(r[1].view(torch.int16), o0[1].view(torch.int16))
+        assert torch.equal(r[2].view(torch.int32), o0[2].view(torch.int32))
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_bounded_wait_gives_up_and_reports(lib, fused):
+    """A wait that gives up (dfs_attn_opts.test_stall_cycles: the MMA warp of
+    every CTA waits on a barrier that nothing arrives at) takes the abort
+    path: the call returns, DFS_FLAG_WAIT_TIMEOUT is raised, no row with a
+    kept block is written (rows with an empty list need no wait and get
+    their zero output), and the context stays usable -- the same launch with
+    the default settings then matches the oracle. (The CTAs of this small
+    launch run split, so both epilogues take the abort path.)"""
+    B, nh, D, blk, N, kcap = 1, 2, 128, 128, 1024, 4
+    nb = -(-N // blk)
+    rng = np.random.default_rng(3)
+    idx, cnt = _lists(rng, B, nh, nb, kcap)
+    cnt[0, 0, 0] = max(1, cnt[0, 0, 0])
+    cnt[0, 1, 3] = 0                            # an empty row
+    s = lib.Shape(B, nh, D, 1, 1, N, blk, 16)
+    g = torch.Generator().manual_seed(5)
+    q, k, v = (torch.randn((B, nh, N, D), generator=g).to(torch.bfloat16) for _ in range(3))
+    qp, kp, vp = q.cuda(), k.cuda(), v.cuda()
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    perm = torch.arange(N, dtype=torch.int32, device="cuda").flip(0).contiguous() if fused else None
+    sentinel = -12345
+    assert lib.dfs_get_error_flags(clear=True) == 0
+    o = torch.full((B, nh, N, D), sentinel, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    lse = None if fused else torch.full((B, nh, N), float("nan"), dtype=torch.float32, device="cuda")
+    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, o, lse, perm=perm, test_stall_cycles=20000)
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == lib.DFS_FLAG_WAIT_TIMEOUT
+    # per token row (curve order) of each head: does its block keep anything?
+    kept = np.repeat(cnt[0] > 0, blk, axis=1)[:, :N]                     # [nh, N]
+    raw = o.view(torch.int16).cpu().numpy()
+    rows = raw.reshape(N, nh, D).transpose(1, 0, 2)[:, perm.cpu().numpy()] if fused else raw[0]
+    assert (rows[kept] == sentinel).all()
+    assert (rows[~kept] == 0).all()
+    if lse is not None:
+        l = lse[0].cpu().numpy()
+        assert np.isnan(l[kept]).all() and np.isneginf(l[~kept]).all()
+    # the same launch with the default settings
+    lib.dfs_sparse_attn_fwd_ex(s, qp, kp, vp, it, ct, kcap, 0.0, o, lse, perm=perm)
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == 0
+    ref, _ = attention.block_sparse_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(), idx, cnt,
+                                              blk)
+    got = o.float().cpu().numpy()
+    if fused:     # raster o[b, perm[i], h, :] = row i of head h, o viewed as [B, N, nh, D]
+        got = got.reshape(B, N, nh, D)[:, perm.long().cpu().numpy()].transpose(0, 2, 1, 3)
+    assert_attn_close(got, ref, "after the abort path")

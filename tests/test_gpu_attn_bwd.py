@@ -152,8 +152,10 @@ def test_rejects_blk64_and_short_workspace(lib):
     small = big[:256]
     with pytest.raises(RuntimeError, match="workspace"):
         lib.dfs_sparse_attn_bwd(s, x, x, x, x, x, lse, idx, cnt, 1, 0.0, x, x, x, small)
+    idx64 = torch.zeros((1, 1, s64.nb, 1), dtype=torch.int32, device="cuda")
+    cnt64 = torch.ones((1, 1, s64.nb), dtype=torch.int32, device="cuda")
     with pytest.raises(RuntimeError, match="unsupported"):
-        lib.dfs_sparse_attn_bwd(s64, x, x, x, x, x, lse, idx, cnt, 1, 0.0, x, x, x, small)
+        lib.dfs_sparse_attn_bwd(s64, x, x, x, x, x, lse, idx64, cnt64, 1, 0.0, x, x, x, small)
 
 
 def test_layer_backward_wan_sampled(lib):

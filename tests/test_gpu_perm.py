@@ -94,10 +94,12 @@ def test_partial_tensors(lib):
                           hilbert.permute_tokens(k.cpu().view(torch.int16).numpy(), operm))
 
 
-@pytest.mark.parametrize("order", ["tile2d", "tile3d"])
+@pytest.mark.parametrize("order", ["tile2d", "tile3d", "hilbert2d"])
 @pytest.mark.parametrize("grid,blk", [((8, 16, 16), 64), ((21, 30, 52), 128), ((3, 5, 7), 64), ((63, 30, 52), 128),
                                       ((33, 45, 80), 128), ((1, 1, 100), 128), ((5, 17, 9), 128)])
-def test_tiled_orders_match_oracle(lib, order, grid, blk):
+def test_tiled_and_2d_orders_match_oracle(lib, order, grid, blk):
+    """Tiled orders and the frame-major 2-D Hilbert order: the index kernel's
+    perm and inv bit-exact against the oracle's enumeration."""
     T, H, W = grid
     N = T * H * W
     perm = torch.empty(N, dtype=torch.int32, device="cuda")

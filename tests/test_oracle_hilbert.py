@@ -171,3 +171,32 @@ def test_tile2d_first_block_by_hand():
     perm, _ = hilbert.make_perm("tile2d", 1, 16, 32, 128)
     assert list(perm[:18]) == list(range(16)) + [32, 33]
     assert perm[127] == 7 * 32 + 15 and perm[128] == 16
+
+
+@pytest.mark.parametrize("T,k", [(1, 1), (3, 2), (2, 4), (5, 5)])
+def test_hilbert2d_frames_follow_the_textbook_curve(T, k):
+    """2-D Hilbert order on T x 2^k x 2^k: frame after frame, each frame in the
+    order of the textbook 2-D Hilbert curve (quadrant-rotation method)."""
+    n = 2 ** k
+    perm, inv = hilbert.make_perm("hilbert2d", T, n, n)
+    ref = [_textbook_2d(n, d) for d in range(n * n)]
+    want = [(t * n + y) * n + x for t in range(T) for (x, y) in ref]
+    assert perm.tolist() == want
+    assert np.array_equal(inv[perm], np.arange(T * n * n))
+
+
+@pytest.mark.parametrize("T,H,W", [(3, 5, 7), (2, 30, 52), (4, 45, 80), (2, 1, 9), (3, 6, 2)])
+def test_hilbert2d_is_frame_major_and_continuous_in_frames(T, H, W):
+    perm, inv = hilbert.make_perm("hilbert2d", T, H, W)
+    P = H * W
+    assert np.array_equal(np.sort(perm), np.arange(T * P)) and np.array_equal(inv[perm], np.arange(T * P))
+    t, r = np.divmod(perm, P)
+    assert np.array_equal(t, np.repeat(np.arange(T), P))          # whole frames, in time order
+    frames = r.reshape(T, P)
+    assert (frames == frames[0]).all()                            # the same path in every frame
+    h, w = np.divmod(frames[0], W)
+    st = np.abs(np.diff(np.stack([h, w], 1), axis=0))
+    if P > 1:
+        assert st.max() == 1                                      # each step to a touching cell
+    if H % 2 == 0 and W % 2 == 0:
+        assert st.sum(axis=1).max() == 1                          # even sides: face steps only
