@@ -54,12 +54,6 @@
 #ifndef DFS_ATTN_EXP2_EMU
 #define DFS_ATTN_EXP2_EMU 0
 #endif
-// 1: with 128-key blocks, S(j+1) is formed in two 64-key halves, the upper
-// one (TMEM columns that P(j) does not occupy) as soon as the softmax has
-// read S(j), the lower one after P.V(j) has read P(j).
-#ifndef DFS_ATTN_EARLY_S
-#define DFS_ATTN_EARLY_S 0
-#endif
 
 namespace {
 
@@ -91,7 +85,7 @@ struct Cfg {
 struct __align__(8) Barriers {
   uint64_t q_full[2];
   uint64_t kv_full[kRing], kv_empty[kRing];
-  uint64_t s_full[2], s_read[2], p_half[2], p_full[2], o_final[2];
+  uint64_t s_full[2], p_half[2], p_full[2], o_final[2];
   uint64_t mma_done;
   uint64_t stall;          // nothing ever arrives here (the abort-path test)
   uint32_t tmem_base;
@@ -109,21 +103,6 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t d
     const uint64_t oa = (uint64_t)(((kk >> 2) * (kQRows * 128) + (kk & 3) * 32) >> 4);
     const uint64_t ob = (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
     mma_ss_warp(d_tmem, dq + oa, dk + ob, idesc, kk > 0 ? 1u : 0u);
-  }
-}
-
-// One 64-key half of S = Q K^T (keys 64 h .. 64 h + 63 of the tile, into
-// TMEM columns d_tmem + 0 .. 63): K rows 64 h .. start 64 h * 128 bytes into
-// each 128-byte-wide slab of the tile.
-template <int D, int BLK>
-__device__ __forceinline__ void issue_s_half(uint32_t d_tmem, uint64_t dq, uint64_t dk, int h) {
-  constexpr uint32_t idesc = idesc_bf16_f32(kQRows, 64, 0);
-  const uint64_t row0 = (uint64_t)((h * 64 * 128) >> 4);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t oa = (uint64_t)(((kk >> 2) * (kQRows * 128) + (kk & 3) * 32) >> 4);
-    const uint64_t ob = (uint64_t)(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
-    mma_ss_warp(d_tmem, dq + oa, dk + ob + row0, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -218,7 +197,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->q_full[x], 1);
       mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->s_read[x], 4);
       mbar_init(&bars->p_half[x], 4);
       mbar_init(&bars->p_full[x], 4);
       mbar_init(&bars->o_final[x], 1);
@@ -322,9 +300,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         prefetch_tensor_map(&tm_v);
       }
       // Same step order as the MMA issuer: step -1 loads K_A(0), K_B(0); step
-      // j loads, per slot, V(j) and then K(j+1) (with the early S halves:
-      // K(j+1) first, its upper half is read before P.V(j)).
-      constexpr bool kEarly = DFS_ATTN_EARLY_S && BLK == 128;
+      // j loads, per slot, V(j) and then K(j+1).
       int t = 0;  // ring tiles loaded so far
       bool ok = true;
       for (int step = -1; step < jmax && ok; ++step) {
@@ -333,8 +309,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int nx = n[x];
           if (step >= nx) continue;
 #pragma unroll 1
-          for (int kk2 = 0; kk2 < 2; ++kk2) {
-            const int kind = kEarly ? 1 - kk2 : kk2;  // 0: V(step), 1: K(step + 1)
+          for (int kind = 0; kind < 2; ++kind) {      // 0: V(step), 1: K(step + 1)
             const int jj = kind == 0 ? step : step + 1;
             if (jj < 0 || jj >= nx) continue;
             const int st = t % kRing;
@@ -383,40 +358,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int x = 0; x < 2; ++x) {
           const int nx = n[x];
           if (step >= nx) continue;
-          if (DFS_ATTN_EARLY_S && BLK == 128 && step >= 0) {
-            // ring order: K(step + 1) [stage tk], then V(step) [stage tv]
-            const bool more = step + 1 < nx;
-            const int tk = t, tv = more ? t + 1 : t;
-            const uint64_t dqx = dq + (uint64_t)((x * C::kQBytes) >> 4);
-            const uint64_t dks = dk + (uint64_t)(((tk % kRing) * C::kTileBytes) >> 4);
-            const uint32_t s_tm = tmem + C::s_col(x);
-            if (more) {
-              // keys 64-127 of S(step + 1) go to columns P(step) leaves free,
-              // once the softmax has read S(step)
-              if (!mbar_wait_bounded(&bars->s_read[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-              if (!mbar_wait_bounded(&bars->kv_full[tk % kRing], (uint32_t)((tk / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-              tc_fence_after();
-              issue_s_half<D, BLK>(s_tm + 64, dqx, dks, 1);
-            }
-            const uint64_t dvs = dv + (uint64_t)(((tv % kRing) * C::kTileBytes) >> 4);
-            if (!mbar_wait_bounded(&bars->p_half[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-            tc_fence_after();
-            if (!mbar_wait_bounded(&bars->kv_full[tv % kRing], (uint32_t)((tv / kRing) & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-            issue_pv<D, BLK, 0, BLK / 32>(tmem + C::o_col(x), s_tm, dvs, step > 0);
-            if (!mbar_wait_bounded(&bars->p_full[x], (uint32_t)(step & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv<D, BLK, BLK / 32, BLK / 16>(tmem + C::o_col(x), s_tm, dvs, true);
-            mma_commit_warp(&bars->kv_empty[tv % kRing]);
-            if (more) {
-              issue_s_half<D, BLK>(s_tm, dqx, dks, 0);   // keys 0-63, over P(step) once P.V(step) has read it
-              mma_commit_warp(&bars->s_full[x]);
-              mma_commit_warp(&bars->kv_empty[tk % kRing]);
-            } else {
-              mma_commit_warp(&bars->o_final[x]);
-            }
-            t += more ? 2 : 1;
-            continue;
-          }
           if (step >= 0) {
             // P_X was written by other threads with tcgen05.st: order this
             // thread's MMAs after their arrival. (TMA-filled tiles need no
@@ -490,12 +431,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[e]);
       }
       tmem_wait_ld();
-      if (DFS_ATTN_EARLY_S && BLK == 128) {
-        // S(j) is in registers: its columns may take the next S
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_read[x]);
-      }
       if (list[j] == nb - 1 && rem < BLK) {
 #pragma unroll
         for (int e = 0; e < BLK; ++e)
