@@ -161,7 +161,8 @@ def test_rejects_blk64_and_short_workspace(lib):
 def test_layer_backward_wan_sampled(lib):
     """Wan-shaped layer end to end: forward, then backward through
     DfsLayer (dO reordered, gradients scattered back to raster order);
-    dQ checked on sampled query blocks, dK/dV on sampled key blocks (each
+    dQ, dK and dV on every row of the first head (the oracle's whole-head
+    gradients), and on sampled blocks of the last head (dK/dV of a key block
     from all query blocks that keep it), by the oracle in curve order."""
     import synth
     import block_sparse_attention_36_b200 as bsa
@@ -197,6 +198,11 @@ def test_layer_backward_wan_sampled(lib):
     _check((np.concatenate(got_q), np.concatenate(got_kv)[:, :wl.D], np.concatenate(got_kv)[:, wl.D:]),
            (np.concatenate(ref_q), np.concatenate(ref_kv)[:, :wl.D], np.concatenate(ref_kv)[:, wl.D:]),
            "Wan layer sampled")
+    # every row of head 0: the oracle's gradients of the whole head
+    cur = [x[0, perm, 0, :].double().numpy()[None, None] for x in (qkv["q"], qkv["k"], qkv["v"], dout)]
+    rq, rk, rv = attention.block_sparse_attention_bwd(*cur, idx[:, :1], cnt[:, :1], wl.blk)
+    got = tuple(x.cpu()[0, perm, 0, :].float().numpy() for x in (dq, dk, dv))
+    _check(got, (rq[0, 0], rk[0, 0], rv[0, 0]), "Wan layer, every row of head 0")
 
 
 def test_layer_backward_hunyuan_sampled(lib):
