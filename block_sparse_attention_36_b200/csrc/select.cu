@@ -100,13 +100,14 @@ select_scores_kernel(const float* __restrict__ scores, int rows, int nb, int mod
   }
   int32_t* out = kv_idx + row * (long long)kcap;
   int kept;
-  uint32_t K;
-  int ties;
-  int take = 0;  // number of blocks to keep
+  uint32_t K = 0u;
+  int ties = 0;
+  bool cut_known = false;  // K and ties already found (threshold)
+  int take = 0;            // number of blocks to keep
   if (mode == DFS_SEL_TOPK) {
     take = min(k, nb);
   } else {
-    // threshold: smallest best-ranked prefix with mass >= tau * Z
+    // threshold: smallest best-ranked prefix with mass >= tau * Z, at most cap
     float m = -INFINITY;
 #pragma unroll
     for (int s = 0; s < S; ++s) m = fmaxf(m, sc[s]);
@@ -120,57 +121,91 @@ select_scores_kernel(const float* __restrict__ scores, int rows, int nb, int mod
     }
     z = warp_sum(z);
     const float target = tau * z;
-    // Largest key value K with mass(key >= K) >= target.
-    uint32_t KK = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = KK | (1u << bit);
-      float ms = 0.f;
+    const int capn = min(cap, nb);
+    if (capn >= 1 && capn < nb) {
+      // The cap first: the capn best blocks are every key above the capn-th
+      // largest key Kc plus the first ties at Kc. If they hold less than the
+      // target, the prefix the rule asks for is longer and the cap decides.
+      const uint32_t Kc = kth_largest_key<S>(key, valid, capn);
+      uint32_t cg = 0;
+      float mg = 0.f, pe = 0.f;
 #pragma unroll
-      for (int s = 0; s < S; ++s) ms += (valid[s] && key[s] >= cand) ? p[s] : 0.f;
-      ms = warp_sum(ms);
-      if (ms >= target) KK = cand;
+      for (int s = 0; s < S; ++s) {
+        if (valid[s] && key[s] > Kc) { cg++; mg += p[s]; }
+        if (valid[s] && key[s] == Kc) pe = p[s];
+      }
+      cg = __reduce_add_sync(0xffffffffu, cg);
+      mg = warp_sum(mg);
+      pe = warp_max(pe);
+      float acc = mg;
+      for (int u = (int)cg; u < capn; ++u) acc += pe;
+      if (acc < target) {
+        take = capn;
+        K = Kc;
+        ties = capn - (int)cg;
+        cut_known = true;
+      }
     }
-    // Blocks strictly above the cut, their mass, and the tie value at the cut.
-    uint32_t cgt = 0, ceq = 0;
-    float mgt = 0.f, peq = 0.f;
+    if (!cut_known) {
+      // Largest key value KK with mass(key >= KK) >= target (a key of the row:
+      // the mass only changes at key values).
+      uint32_t KK = 0;
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = KK | (1u << bit);
+        float ms = 0.f;
 #pragma unroll
-    for (int s = 0; s < S; ++s) {
-      if (valid[s] && key[s] > KK) { cgt++; mgt += p[s]; }
-      if (valid[s] && key[s] == KK) { ceq++; peq = p[s]; }
+        for (int s = 0; s < S; ++s) ms += (valid[s] && key[s] >= cand) ? p[s] : 0.f;
+        ms = warp_sum(ms);
+        if (ms >= target) KK = cand;
+      }
+      // Blocks strictly above the cut, their mass, and the tie value at the cut.
+      uint32_t cgt = 0, ceq = 0;
+      float mgt = 0.f, peq = 0.f;
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        if (valid[s] && key[s] > KK) { cgt++; mgt += p[s]; }
+        if (valid[s] && key[s] == KK) { ceq++; peq = p[s]; }
+      }
+      cgt = __reduce_add_sync(0xffffffffu, cgt);
+      ceq = __reduce_add_sync(0xffffffffu, ceq);
+      mgt = warp_sum(mgt);
+      peq = warp_max(peq);
+      // mgt < target by the choice of KK (the warp sums are monotone in the
+      // set summed). Equal scores carry equal mass: add them one at a time,
+      // lowest column first, until the target is reached.
+      int t = 0;
+      float acc = mgt;
+      while (t < (int)ceq && acc < target) { acc += peq; ++t; }
+      take = max(1, (int)cgt + t);   // the shortest prefix holds at least one block
+      take = min(take, capn);
+      if (t >= 1 && take == (int)cgt + t) {
+        // the cut is KK itself: every key above it and t of its ties
+        K = KK;
+        ties = t;
+        cut_known = true;
+      }
     }
-    cgt = __reduce_add_sync(0xffffffffu, cgt);
-    ceq = __reduce_add_sync(0xffffffffu, ceq);
-    mgt = warp_sum(mgt);
-    peq = warp_max(peq);
-    // mgt < target by the choice of KK (the warp sums are monotone in the
-    // set summed). Equal scores carry equal mass: add them one at a time,
-    // lowest column first, until the target is reached.
-    int t = 0;
-    float acc = mgt;
-    while (t < (int)ceq && acc < target) { acc += peq; ++t; }
-    take = max(1, (int)cgt + t);   // the shortest prefix holds at least one block
-    take = min(take, min(cap, nb));
   }
   if (take <= 0) {
     kept = 0;
   } else if (take >= nb) {
     // keep all columns
-    K = 0u;
-    ties = nb;
     bool all[S];
 #pragma unroll
     for (int s = 0; s < S; ++s) all[s] = valid[s];
     uint32_t zk[S];
 #pragma unroll
     for (int s = 0; s < S; ++s) zk[s] = 0u;
-    kept = emit_row<S>(zk, all, K, ties, out, kcap, lane);
+    kept = emit_row<S>(zk, all, 0u, nb, out, kcap, lane);
   } else {
-    K = kth_largest_key<S>(key, valid, take);
-    uint32_t cgt = 0;
+    if (!cut_known) {
+      K = kth_largest_key<S>(key, valid, take);
+      uint32_t cgt = 0;
 #pragma unroll
-    for (int s = 0; s < S; ++s) cgt += (valid[s] && key[s] > K) ? 1u : 0u;
-    cgt = __reduce_add_sync(0xffffffffu, cgt);
-    ties = take - (int)cgt;
+      for (int s = 0; s < S; ++s) cgt += (valid[s] && key[s] > K) ? 1u : 0u;
+      cgt = __reduce_add_sync(0xffffffffu, cgt);
+      ties = take - (int)cgt;
+    }
     kept = emit_row<S>(key, valid, K, ties, out, kcap, lane);
   }
   if (lane == 0) {
