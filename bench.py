@@ -55,9 +55,10 @@ ATTN_TRAFFIC = {"wan_1p3b_layer": (298_866_176 + 83_991_552, "055f4a481e84b06c")
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 
-# dram read + write of one backward call (all its launches) on the Wan layer,
-# from a one-pass ncu capture of these sources
-BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_816_448 + 262_639_360, "a64bc91715fa78dd")}
+# dram read + write of one backward call (its prep, list and gradient
+# launches), from a one-pass ncu capture of these sources
+BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_286_528 + 263_357_952, "d6d9083fa2066969"),
+               "hunyuan_layer": (18_739_300_352 + 2_202_705_152, "d6d9083fa2066969")}
 BWD_SOURCES = ("attn_bwd.cu", "sm100_ptx.cuh", "common.cuh", "tmap.cuh")
 
 

@@ -20,9 +20,11 @@
 // transposed lists through a bitset of the kept mask.
 // Both passes: warp 0 loads tiles with TMA (128-byte swizzle, no multicast),
 // warp 1 owns tensor memory and issues the tcgen05 MMAs from one elected
-// lane, warp 2 stages the list, warps 4-11 are two warpgroups that each take
-// one half of the 128 columns of the score tiles (one TMEM lane per row) and
-// write P or dS back as bf16 into the columns they have read. Keys beyond N
+// lane, warp 2 stages (dQ) or counts (dK/dV) the list, warps 4-11 are two
+// warpgroups that each take one half of the 128 columns of the score tiles
+// (one TMEM lane per row). dS goes back as bf16 into the tensor-memory
+// columns it was read from; P^T of the dK/dV pass goes to a shared-memory
+// tile instead, so that the next S^T need not wait for dV. Keys beyond N
 // have zero K and V rows (TMA fill), so they add nothing to dQ, and their dK,
 // dV rows are not stored. Every mbarrier wait is bounded (timeout flag,
 // early return); copies and MMAs in flight are drained before tensor memory
@@ -49,19 +51,11 @@ template <int D>
 struct Bw {
   static constexpr int kChunks = D / 64;          // 128-byte column slabs per row
   static constexpr int kTile = kBlk * D * 2;      // one 128-row tile
-  // dQ pass shared memory: the K/V ring only
+  // dQ pass: shared memory holds the K/V ring only
   static constexpr int kRingOff = 0;
   static constexpr int kQBarOff = kRingOff + kRing * kTile;
-  // dK/dV pass shared memory: K, V, then two stages of
-  // {Q, dO, -lse log2 e [128], -Delta [128]}
-  static constexpr int kKOff = 0;
-  static constexpr int kVOff = kTile;
-  static constexpr int kStageOff = 2 * kTile;
-  static constexpr int kStageBytes = 2 * kTile + 1024;
-  static constexpr int kKVBarOff = kStageOff + 2 * kStageBytes;
   // tensor memory columns
-  static constexpr int kS = 0, kDP = 128, kDQ = 256, kQT = 256 + D, kDOT = 256 + D + D / 2;  // dQ pass
-  static constexpr int kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D;  // dK/dV pass
+  static constexpr int kS = 0, kDP = 128, kDQ = 256, kQT = 256 + D, kDOT = 256 + D + D / 2;
 };
 
 // Untiled bulk copy global -> shared completing on an mbarrier, from
@@ -492,39 +486,92 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 }
 
 // ------------------------------------------------------------ dK/dV pass
+// Shared memory: K, V, two stages of {Q, dO, -lse log2 e [128], -Delta [128]},
+// the P^T tile; then the tensor memory columns.
+template <int D>
+struct BwKV {
+  static constexpr int kTile = kBlk * D * 2;        // one 128-row Q / dO / K / V tile
+  static constexpr int kPtBytes = kBlk * kBlk * 2;  // P^T: 128 keys x 128 queries, bf16
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kTile;
+  static constexpr int kStageOff = 2 * kTile;
+  static constexpr int kStageBytes = 2 * kTile + 1024;
+  static constexpr int kPtOff = kStageOff + 2 * kStageBytes;
+  static constexpr int kTiles = kPtOff + kPtBytes;  // everything that needs 1024-byte alignment
+  static constexpr int kST_col = 0, kDPT_col = 128, kDV_col = 256, kDK_col = 256 + D;  // tensor memory
+};
+
 struct __align__(8) BarsKV {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
-  uint64_t st_full, dpt_full, p_ready, ds_ready, kv_final, mma_done;
+  uint64_t st_full, dpt_full, s_read, p_ready, p_free, ds_ready, kv_final, mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int n_q;
 };
 
-// Per query block i of the transposed list the P/dS warps run two phases:
-// A forms P^T(i) from S^T(i) (the exponentials) and hands it to dV(i);
-// B forms dS^T(i) once dP^T(i) is there and hands it to dK(i). MMA order:
-// S^T(0) dP^T(0), then per i: [P^T(i)] dV(i) S^T(i+1) [dS^T(i)] dK(i)
-// dP^T(i+1). S^T(i+1) reuses the columns of P^T(i) after dV(i) and
-// dP^T(i+1) those of dS^T(i) after dK(i) (in-order MMAs), so phase A of
-// i+1 overlaps dK(i) and dP^T(i+1), and phase B of i overlaps dV(i) and
-// S^T(i+1).
+// The shared-memory window of a CTA: the 1024-byte-aligned tiles and the
+// barriers, placed in whichever of three ways fits
+// tiles + sizeof(BarsKV) + 1008 bytes from any 16-byte-aligned base.
+struct SmemKV {
+  uint8_t* tiles;
+  BarsKV* bars;
+};
+template <int D>
+__device__ __forceinline__ SmemKV place_smem_kv(uint8_t* raw) {
+  const uint32_t a = smem_addr(raw) & 1023u;
+  SmemKV r;
+  if (a == 0) {
+    r.tiles = raw;
+    r.bars = reinterpret_cast<BarsKV*>(raw + BwKV<D>::kTiles);
+  } else if (a + sizeof(BarsKV) <= 1024u) {
+    r.bars = reinterpret_cast<BarsKV*>(raw);
+    r.tiles = raw + (1024u - a);
+  } else {
+    r.tiles = raw + (1024u - a);
+    r.bars = reinterpret_cast<BarsKV*>(r.tiles + BwKV<D>::kTiles);
+  }
+  return r;
+}
+
+// D (+)= A B with A (128 x 128 bf16, K-major, 128-byte swizzled) and B a
+// 128-row tile read MN-major, both in shared memory.
+template <int D>
+__device__ __forceinline__ void issue_ss_tn(uint32_t d_tmem, uint64_t da, uint64_t db, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBlk, D, 1);
+#pragma unroll
+  for (int kk = 0; kk < kBlk / 16; ++kk) {
+    const uint64_t aoff = (uint64_t)(((kk >> 2) * (kBlk * 128) + (kk & 3) * 32) >> 4);
+    mma_ss_warp(d_tmem, da + aoff, db + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Per query block i of the transposed list the P/dS warps read S^T(i) from
+// tensor memory (and report it read, so that S^T(i+1) can start at once),
+// form P^T(i) into a shared-memory tile for dV(i), then dS^T(i) over dP^T(i)
+// in tensor memory for dK(i). MMA order: S^T(0) dP^T(0), then per i:
+// [S^T(i) read] S^T(i+1) [P^T(i)] dV(i) [dS^T(i)] dK(i) dP^T(i+1). The
+// exponentials of block i overlap S^T(i+1), dK(i-1) and dP^T(i); P^T(i+1)
+// is written once dV(i) has read P^T(i).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const int32_t* __restrict__ q_idx, const int32_t* __restrict__ q_cnt, int N, int nb,
-                     float scale, float scale_log2, const float* __restrict__ nlse,
-                     const float* __restrict__ ndelta, __nv_bfloat16* __restrict__ dk,
-                     __nv_bfloat16* __restrict__ dv) {
-  using C = Bw<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  BarsKV* bars = reinterpret_cast<BarsKV*>(smem + C::kKVBarOff);
-  int32_t* list = reinterpret_cast<int32_t*>(smem + C::kKVBarOff + sizeof(BarsKV));
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const int32_t* __restrict__ q_idx, const int32_t* __restrict__ q_cnt, int N, int nb,
+                        float scale, float scale_log2, const float* __restrict__ nlse,
+                        const float* __restrict__ ndelta, __nv_bfloat16* __restrict__ dk,
+                        __nv_bfloat16* __restrict__ dv) {
+  using C = BwKV<D>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const SmemKV sp = place_smem_kv<D>(smem_raw);
+  uint8_t* smem = sp.tiles;
+  BarsKV* bars = sp.bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int J = blockIdx.x, bh = blockIdx.y;
   volatile int* abort_flag = &bars->abort_flag;
+  const long long col = (long long)bh * nb + J;
+  const int cnt = max(0, min(q_cnt[col], nb));
+  const int32_t* src = q_idx + col * nb;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -534,7 +581,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->dpt_full, 1);
+    mbar_init(&bars->s_read, 8);
     mbar_init(&bars->p_ready, 8);
+    mbar_init(&bars->p_free, 1);
     mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->kv_final, 1);
     mbar_init(&bars->mma_done, 1);
@@ -542,19 +591,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     fence_barrier_init();
   }
   if (warp == 2) {
-    const long long col = (long long)bh * nb + J;
-    const int cnt = max(0, min(q_cnt[col], nb));
-    const int32_t* src = q_idx + col * nb;
-    int base = 0;
+    // valid entries of the list (the producer skips the others in the same order)
+    int valid = 0;
     for (int i0 = 0; i0 < cnt; i0 += 32) {
       const int i = i0 + lane;
       const int Iq = (i < cnt) ? src[i] : -1;
-      const bool ok = (i < cnt) && Iq >= 0 && Iq < nb;
-      const unsigned m = __ballot_sync(0xffffffffu, ok);
-      if (ok) list[base + __popc(m & ((1u << lane) - 1u))] = Iq;
-      base += __popc(m);
+      valid += __popc(__ballot_sync(0xffffffffu, Iq >= 0 && Iq < nb));
     }
-    if (lane == 0) bars->n_q = base;
+    if (lane == 0) bars->n_q = valid;
   }
   if (warp == 1) tmem_alloc(&bars->tmem_base, kTmemCols);
   tc_fence_before();
@@ -575,20 +619,33 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (n > 0) {
       mbar_arrive_expect_tx_warp(&bars->kv_full, 2 * C::kTile);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         tma_load_3d_warp(smem + C::kKOff + c * (kBlk * 128), &tm_k, &bars->kv_full, c * 64, J * kBlk, bh);
         tma_load_3d_warp(smem + C::kVOff + c * (kBlk * 128), &tm_v, &bars->kv_full, c * 64, J * kBlk, bh);
       }
     }
+    // The list is read 32 entries at a time (one per lane); `pend` holds the
+    // lanes of the current group whose entries are valid and not yet used.
+    int g0 = -32;
+    int mine = -1;
+    unsigned pend = 0u;
     int i = 0;
     for (; i < n; ++i) {
+      while (pend == 0u && g0 + 32 < cnt) {
+        g0 += 32;
+        mine = (g0 + lane < cnt) ? src[g0 + lane] : -1;
+        pend = __ballot_sync(0xffffffffu, mine >= 0 && mine < nb);
+      }
+      if (pend == 0u) break;  // cannot happen: n counts the valid entries
+      const int src_lane = __ffs(pend) - 1;
+      pend &= pend - 1u;
+      const int Iq = __shfl_sync(0xffffffffu, mine, src_lane);
       const int st = i & 1;
       if (!mbar_wait_bounded(&bars->q_empty[st], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag, kWaitLimit)) break;
       mbar_arrive_expect_tx_warp(&bars->q_full[st], 2 * C::kTile + 1024);
-      const int Iq = list[i];
       uint8_t* stage = smem + C::kStageOff + st * C::kStageBytes;
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         tma_load_3d_warp(stage + c * (kBlk * 128), &tm_q, &bars->q_full[st], c * 64, Iq * kBlk, bh);
         tma_load_3d_warp(stage + C::kTile + c * (kBlk * 128), &tm_do, &bars->q_full[st], c * 64, Iq * kBlk, bh);
       }
@@ -596,6 +653,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       bulk_load_warp(stage + 2 * C::kTile, nlse + prow, kBlk * 4, &bars->q_full[st]);
       bulk_load_warp(stage + 2 * C::kTile + 512, ndelta + prow, kBlk * 4, &bars->q_full[st]);
     }
+    if (i < n) *abort_flag = 1;
     for (int w = max(0, i - 2); w < i; ++w)
       mbar_wait_timed(&bars->q_full[w & 1], (uint32_t)((w >> 1) & 1), kDrainLimit);
     if (n > 0) mbar_wait_timed(&bars->kv_full, 0, kDrainLimit);
@@ -605,6 +663,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint64_t dv_k = desc_sw128(smem_addr(smem + C::kVOff), 16, 1024);
     const uint64_t st_k = desc_sw128(smem_addr(smem + C::kStageOff), 16, 1024);
     const uint64_t st_mn = desc_sw128(smem_addr(smem + C::kStageOff), kBlk * 128, 1024);
+    const uint64_t pt_k = desc_sw128(smem_addr(smem + C::kPtOff), 16, 1024);
     bool ok = true;
     auto q_off = [](int i) { return (uint64_t)(((i & 1) * C::kStageBytes) >> 4); };
     auto do_off = [](int i) { return (uint64_t)(((i & 1) * C::kStageBytes + C::kTile) >> 4); };
@@ -612,32 +671,36 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ok = mbar_wait_bounded(&bars->kv_full, 0, abort_flag, kWaitLimit) &&
            mbar_wait_bounded(&bars->q_full[0], 0, abort_flag, kWaitLimit);
       if (ok) {
-        issue_nt<D>(tmem + C::kST, dk_k, st_k + q_off(0));     // S^T = K Q^T
+        issue_nt<D>(tmem + C::kST_col, dk_k, st_k + q_off(0));     // S^T = K Q^T
         mma_commit_warp(&bars->st_full);
-        issue_nt<D>(tmem + C::kDPT, dv_k, st_k + do_off(0));   // dP^T = V dO^T
+        issue_nt<D>(tmem + C::kDPT_col, dv_k, st_k + do_off(0));   // dP^T = V dO^T
         mma_commit_warp(&bars->dpt_full);
       }
     }
     for (int i = 0; i < n && ok; ++i) {
-      // P^T(i) and dS^T(i) are written with tcgen05.st by other threads:
-      // order the MMAs that read them after their arrivals.
-      if (!mbar_wait_bounded(&bars->p_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
-      tc_fence_after();
-      issue_tn<D>(tmem + C::kDV, tmem + C::kST, st_mn + do_off(i), i > 0);    // dV += P^T dO
       if (i + 1 < n) {
-        if (!mbar_wait_bounded(&bars->q_full[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1), abort_flag, kWaitLimit)) {
+        // S^T(i) has been read into registers: S^T(i+1) may overwrite it
+        if (!mbar_wait_bounded(&bars->s_read, (uint32_t)(i & 1), abort_flag, kWaitLimit) ||
+            !mbar_wait_bounded(&bars->q_full[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1), abort_flag, kWaitLimit)) {
           ok = false;
           break;
         }
-        issue_nt<D>(tmem + C::kST, dk_k, st_k + q_off(i + 1));
+        tc_fence_after();
+        issue_nt<D>(tmem + C::kST_col, dk_k, st_k + q_off(i + 1));
         mma_commit_warp(&bars->st_full);
       }
+      // P^T(i) was stored by other threads and made visible to the tensor
+      // cores (fence.proxy.async) before their arrivals.
+      if (!mbar_wait_bounded(&bars->p_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
+      issue_ss_tn<D>(tmem + C::kDV_col, pt_k, st_mn + do_off(i), i > 0);   // dV += P^T dO
+      mma_commit_warp(&bars->p_free);
+      // dS^T(i) was written with tcgen05.st by other threads
       if (!mbar_wait_bounded(&bars->ds_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       tc_fence_after();
-      issue_tn<D>(tmem + C::kDK, tmem + C::kDPT, st_mn + q_off(i), i > 0);    // dK += dS^T Q
+      issue_tn<D>(tmem + C::kDK_col, tmem + C::kDPT_col, st_mn + q_off(i), i > 0);    // dK += dS^T Q
       mma_commit_warp(&bars->q_empty[i & 1]);
       if (i + 1 < n) {
-        issue_nt<D>(tmem + C::kDPT, dv_k, st_k + do_off(i + 1));
+        issue_nt<D>(tmem + C::kDPT_col, dv_k, st_k + do_off(i + 1));
         mma_commit_warp(&bars->dpt_full);
       }
     }
@@ -652,6 +715,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int r = sub * 32 + lane;                  // key row in the block
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
     const float2 sc2 = make_float2(scale_log2, scale_log2);
+    // this thread's row of P^T in slab g (queries 64g .. 64g + 63), 128-byte swizzled
+    uint8_t* pt_row = smem + C::kPtOff + g * (kBlk * 128) + (r >> 3) * 1024 + (r & 7) * 128;
+    const int sw = r & 7;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int st = i & 1;
@@ -664,34 +730,49 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tc_fence_after();
       const float* nl = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes + 2 * C::kTile);
       const float* nd = nl + kBlk;
-      const uint32_t s_addr = tmem + lane_base + C::kST + 64 * g;
-      const uint32_t p_addr = tmem + lane_base + C::kDPT + 64 * g;
-      // phase A: P^T = 2^(S^T scale log2 e - lse log2 e), kept in fp32 for phase B
+      const uint32_t s_addr = tmem + lane_base + C::kST_col + 64 * g;
+      const uint32_t p_addr = tmem + lane_base + C::kDPT_col + 64 * g;
+      // phase A: S^T(i) into registers, then P^T = 2^(S^T scale log2 e - lse log2 e)
+      uint32_t sr[64];
+      {
+        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tmem_ld32(s_addr, s0);
+        tmem_ld32(s_addr + 32, s1);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_read);
+      // dV(i-1) has read P^T(i-1)
+      if (i > 0 && !mbar_wait_bounded(&bars->p_free, (uint32_t)((i - 1) & 1), abort_flag, kWaitLimit)) {
+        ok = false;
+        break;
+      }
       float pv[64];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t sr[32], po[16];
-        tmem_ld32(s_addr + 32 * c, sr);
-        // this chunk's 32 constants, loaded while the tensor-memory load is in flight
         float4 nl4[8];
 #pragma unroll
         for (int v = 0; v < 8; ++v) nl4[v] = *reinterpret_cast<const float4*>(nl + 64 * g + 32 * c + 4 * v);
-        tmem_wait_ld();
+        uint32_t po[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 nl2 = (e & 1) ? make_float2(nl4[e >> 1].z, nl4[e >> 1].w) : make_float2(nl4[e >> 1].x, nl4[e >> 1].y);
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sc2, nl2);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[32 * c + 2 * e]), __uint_as_float(sr[32 * c + 2 * e + 1])), sc2, nl2);
           pv[32 * c + 2 * e] = ex2(x.x);
           pv[32 * c + 2 * e + 1] = ex2(x.y);
           po[e] = pack_bf16x2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]);
         }
-        tmem_st16(s_addr + 16 * c, po);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(pt_row + (((4 * c + v) ^ sw) << 4)) =
+              make_uint4(po[4 * v], po[4 * v + 1], po[4 * v + 2], po[4 * v + 3]);
       }
-      tmem_wait_st();
-      tc_fence_before();
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
-      // phase B: dS^T = P^T (dP^T - Delta)
+      // phase B: dS^T = P^T (dP^T - Delta), packed over dP^T(i)
       if (!mbar_wait_bounded(&bars->dpt_full, (uint32_t)(i & 1), abort_flag, kWaitLimit)) {
         ok = false;
         break;
@@ -728,7 +809,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     for (int c = 0; c < D / 64; ++c) {
       uint32_t raw[32];
       if (n > 0 && ok) {
-        tmem_ld32(tmem + lane_base + C::kDV + (D / 2) * g + 32 * c, raw);
+        tmem_ld32(tmem + lane_base + C::kDV_col + (D / 2) * g + 32 * c, raw);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -736,7 +817,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       store_row32(dv + roff + 32 * c, raw, 1.0f, store);
       if (n > 0 && ok) {
-        tmem_ld32(tmem + lane_base + C::kDK + (D / 2) * g + 32 * c, raw);
+        tmem_ld32(tmem + lane_base + C::kDK_col + (D / 2) * g + 32 * c, raw);
         tmem_wait_ld();
       }
       store_row32(dk + roff + 32 * c, raw, scale, store);
@@ -795,7 +876,10 @@ int launch_bwd(const dfs::Dims& d, const void* qp, const void* kp, const void* v
   // the scheduler never places two.
   const size_t min_smem = 120 * 1024;
   size_t smem_q = 1024 + C::kQBarOff + sizeof(BarsQ) + (size_t)max_list * 4;
-  size_t smem_kv = 1024 + C::kKVBarOff + sizeof(BarsKV) + (size_t)nb * 4;
+  // tiles + the worst case of place_smem_kv: a base 16 bytes past a
+  // 1024-byte boundary puts the barriers below the tiles, 1008 bytes on
+  static_assert(2 * sizeof(BarsKV) <= 1008, "barrier block too large");
+  size_t smem_kv = (size_t)BwKV<D>::kTiles + 1008;
   if (smem_q > 232448 || smem_kv > 232448 || (size_t)8 * nw * 4 > 48 * 1024) return DFS_ERR_UNSUPPORTED;
   smem_q = smem_q < min_smem ? min_smem : smem_q;
   smem_kv = smem_kv < min_smem ? min_smem : smem_kv;
