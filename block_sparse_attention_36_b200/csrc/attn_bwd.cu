@@ -503,7 +503,8 @@ struct BwKV {
 
 struct __align__(8) BarsKV {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t qq_full[2], qq_empty[2];  // Q and the two per-query constant rows of a stage
+  uint64_t qd_full[2], qd_empty[2];  // dO of a stage
   uint64_t st_full, dpt_full, s_read, p_ready, p_free, ds_ready, kv_final, mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -576,8 +577,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->qq_full[s], 1);
+      mbar_init(&bars->qq_empty[s], 1);
+      mbar_init(&bars->qd_full[s], 1);
+      mbar_init(&bars->qd_empty[s], 1);
     }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->dpt_full, 1);
@@ -629,7 +632,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     int g0 = -32;
     int mine = -1;
     unsigned pend = 0u;
-    int i = 0;
+    int i = 0, nq = 0, nd = 0;  // blocks whose Q / dO copies were issued
     for (; i < n; ++i) {
       while (pend == 0u && g0 + 32 < cnt) {
         g0 += 32;
@@ -641,21 +644,32 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       pend &= pend - 1u;
       const int Iq = __shfl_sync(0xffffffffu, mine, src_lane);
       const int st = i & 1;
-      if (!mbar_wait_bounded(&bars->q_empty[st], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag, kWaitLimit)) break;
-      mbar_arrive_expect_tx_warp(&bars->q_full[st], 2 * C::kTile + 1024);
+      const uint32_t ep = (uint32_t)(((i >> 1) & 1) ^ 1);
       uint8_t* stage = smem + C::kStageOff + st * C::kStageBytes;
+      // dO first: its half of the stage is free once dV(i-2) is done, the
+      // Q half (with the constants) only once dK(i-2) is
+      if (!mbar_wait_bounded(&bars->qd_empty[st], ep, abort_flag, kWaitLimit)) break;
+      mbar_arrive_expect_tx_warp(&bars->qd_full[st], C::kTile);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d_warp(stage + c * (kBlk * 128), &tm_q, &bars->q_full[st], c * 64, Iq * kBlk, bh);
-        tma_load_3d_warp(stage + C::kTile + c * (kBlk * 128), &tm_do, &bars->q_full[st], c * 64, Iq * kBlk, bh);
-      }
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d_warp(stage + C::kTile + c * (kBlk * 128), &tm_do, &bars->qd_full[st], c * 64, Iq * kBlk, bh);
+      nd = i + 1;
+      if (!mbar_wait_bounded(&bars->qq_empty[st], ep, abort_flag, kWaitLimit)) break;
+      mbar_arrive_expect_tx_warp(&bars->qq_full[st], C::kTile + 1024);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d_warp(stage + c * (kBlk * 128), &tm_q, &bars->qq_full[st], c * 64, Iq * kBlk, bh);
       const long long prow = (long long)bh * padded + (long long)Iq * kBlk;
-      bulk_load_warp(stage + 2 * C::kTile, nlse + prow, kBlk * 4, &bars->q_full[st]);
-      bulk_load_warp(stage + 2 * C::kTile + 512, ndelta + prow, kBlk * 4, &bars->q_full[st]);
+      bulk_load_warp(stage + 2 * C::kTile, nlse + prow, kBlk * 4, &bars->qq_full[st]);
+      bulk_load_warp(stage + 2 * C::kTile + 512, ndelta + prow, kBlk * 4, &bars->qq_full[st]);
+      nq = i + 1;
     }
     if (i < n) *abort_flag = 1;
-    for (int w = max(0, i - 2); w < i; ++w)
-      mbar_wait_timed(&bars->q_full[w & 1], (uint32_t)((w >> 1) & 1), kDrainLimit);
+    // copies still in flight: at most the last two of each kind
+    for (int w = max(0, nd - 2); w < nd; ++w)
+      mbar_wait_timed(&bars->qd_full[w & 1], (uint32_t)((w >> 1) & 1), kDrainLimit);
+    for (int w = max(0, nq - 2); w < nq; ++w)
+      mbar_wait_timed(&bars->qq_full[w & 1], (uint32_t)((w >> 1) & 1), kDrainLimit);
     if (n > 0) mbar_wait_timed(&bars->kv_full, 0, kDrainLimit);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -669,10 +683,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto do_off = [](int i) { return (uint64_t)(((i & 1) * C::kStageBytes + C::kTile) >> 4); };
     if (n > 0) {
       ok = mbar_wait_bounded(&bars->kv_full, 0, abort_flag, kWaitLimit) &&
-           mbar_wait_bounded(&bars->q_full[0], 0, abort_flag, kWaitLimit);
+           mbar_wait_bounded(&bars->qq_full[0], 0, abort_flag, kWaitLimit);
       if (ok) {
         issue_nt<D>(tmem + C::kST_col, dk_k, st_k + q_off(0));     // S^T = K Q^T
         mma_commit_warp(&bars->st_full);
+        ok = mbar_wait_bounded(&bars->qd_full[0], 0, abort_flag, kWaitLimit);
+      }
+      if (ok) {
         issue_nt<D>(tmem + C::kDPT_col, dv_k, st_k + do_off(0));   // dP^T = V dO^T
         mma_commit_warp(&bars->dpt_full);
       }
@@ -681,7 +698,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (i + 1 < n) {
         // S^T(i) has been read into registers: S^T(i+1) may overwrite it
         if (!mbar_wait_bounded(&bars->s_read, (uint32_t)(i & 1), abort_flag, kWaitLimit) ||
-            !mbar_wait_bounded(&bars->q_full[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1), abort_flag, kWaitLimit)) {
+            !mbar_wait_bounded(&bars->qq_full[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1), abort_flag, kWaitLimit)) {
           ok = false;
           break;
         }
@@ -694,12 +711,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!mbar_wait_bounded(&bars->p_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       issue_ss_tn<D>(tmem + C::kDV_col, pt_k, st_mn + do_off(i), i > 0);   // dV += P^T dO
       mma_commit_warp(&bars->p_free);
+      mma_commit_warp(&bars->qd_empty[i & 1]);                                // dO(i) read
       // dS^T(i) was written with tcgen05.st by other threads
       if (!mbar_wait_bounded(&bars->ds_ready, (uint32_t)(i & 1), abort_flag, kWaitLimit)) { ok = false; break; }
       tc_fence_after();
       issue_tn<D>(tmem + C::kDK_col, tmem + C::kDPT_col, st_mn + q_off(i), i > 0);    // dK += dS^T Q
-      mma_commit_warp(&bars->q_empty[i & 1]);
+      mma_commit_warp(&bars->qq_empty[i & 1]);                                // Q(i), constants read
       if (i + 1 < n) {
+        if (!mbar_wait_bounded(&bars->qd_full[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1), abort_flag, kWaitLimit)) {
+          ok = false;
+          break;
+        }
         issue_nt<D>(tmem + C::kDPT_col, dv_k, st_k + do_off(i + 1));
         mma_commit_warp(&bars->dpt_full);
       }
@@ -721,9 +743,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int st = i & 1;
-      // q_full: the stage's -lse and -Delta rows, written by the bulk copy
+      // qq_full: the stage's -lse and -Delta rows, written by the bulk copy
       if (!mbar_wait_bounded(&bars->st_full, (uint32_t)(i & 1), abort_flag, kWaitLimit) ||
-          !mbar_wait_bounded(&bars->q_full[st], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimit)) {
+          !mbar_wait_bounded(&bars->qq_full[st], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimit)) {
         ok = false;
         break;
       }
