@@ -512,8 +512,10 @@ struct __align__(8) BarsKV {
 };
 
 // The shared-memory window of a CTA: the 1024-byte-aligned tiles and the
-// barriers, placed in whichever of three ways fits
-// tiles + sizeof(BarsKV) + 1008 bytes from any 16-byte-aligned base.
+// barriers, placed in whichever of three ways fits tiles + 1008 bytes from
+// any 16-byte-aligned base. The window is declared 1024-byte aligned, so
+// the first way is the one taken; the others keep the layout in bounds
+// should a base ever arrive less aligned.
 struct SmemKV {
   uint8_t* tiles;
   BarsKV* bars;
@@ -563,7 +565,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         const float* __restrict__ ndelta, __nv_bfloat16* __restrict__ dk,
                         __nv_bfloat16* __restrict__ dv) {
   using C = BwKV<D>;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const SmemKV sp = place_smem_kv<D>(smem_raw);
   uint8_t* smem = sp.tiles;
   BarsKV* bars = sp.bars;
