@@ -57,8 +57,8 @@ ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa
 
 # dram read + write of one backward call (its prep, list and gradient
 # launches), from a one-pass ncu capture of these sources
-BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_026_176 + 262_441_472, "ff4f39b43d4953e9"),
-               "hunyuan_layer": (19_861_653_248 + 2_200_965_376, "ff4f39b43d4953e9")}
+BWD_TRAFFIC = {"wan_1p3b_layer": (1_007_642_880 + 262_761_728, "b85a7531aeaa6e3b"),
+               "hunyuan_layer": (19_747_298_560 + 2_204_054_528, "b85a7531aeaa6e3b")}
 BWD_SOURCES = ("attn_bwd.cu", "sm100_ptx.cuh", "common.cuh", "tmap.cuh")
 
 

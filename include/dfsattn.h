@@ -255,7 +255,8 @@ typedef struct {
    * has SMs) into one-row CTAs that give each half of the row's kept list
    * to one of their two tiles and merge the two partial softmax states --
    * the same rows in about half the time. The merged rows differ from the
-   * unsplit ones by rounding only. Nonzero: every CTA takes two rows.
+   * unsplit ones by rounding only (the halves are those of the counted
+   * list, invalid entries included). Nonzero: every CTA takes two rows.
    * dfs_sparse_attn_fwd and dfs_sparse_attn_lvsa_fwd use the default.      */
   int no_tail_split;
   /* test_stall_cycles: testing only, 0 in normal use. Nonzero makes every

@@ -113,6 +113,62 @@ def test_empty_rows_and_unused_keys(lib):
     _check((dq, dk, dv), ref, "empty rows")
 
 
+def test_invalid_entries_are_skipped_and_flagged(lib):
+    """Entries outside [0, nb) inside the counted part of a list are skipped
+    by both passes (the dQ pass reads the caller's lists, in groups of 32)
+    and raise DFS_FLAG_BAD_KV_INDEX; the gradients equal those of the lists
+    without them."""
+    B, nh, D, N = 1, 2, 128, 5000
+    nb = -(-N // 128)                      # 40 blocks: lists span two groups of 32
+    kcap = nb
+    rng = np.random.default_rng(11)
+    idx = np.full((B, nh, nb, kcap), -1, dtype=np.int32)
+    cnt = np.zeros((B, nh, nb), dtype=np.int32)
+    clean_idx = np.full_like(idx, -1)
+    clean_cnt = np.zeros_like(cnt)
+    for h in range(nh):
+        for I in range(nb):
+            c = int(rng.integers(1, 38))   # with up to 3 invalid entries: at most kcap = 40
+            js = list(np.sort(rng.choice(nb, size=c, replace=False)))
+            row = list(js)
+            for pos, bad in ((0, -1), (len(row) // 2, nb), (len(row), nb + 7)):
+                if I % 3 == h % 3:
+                    row.insert(pos, bad)
+            idx[0, h, I, :len(row)] = row
+            cnt[0, h, I] = len(row)
+            clean_idx[0, h, I, :c] = js
+            clean_cnt[0, h, I] = c
+    q, k, v, do = _inputs(B, nh, N, D, 21)
+    s = lib.Shape(B, nh, D, 1, 1, N, 128, 16)
+    dev = [t.cuda() for t in (q, k, v, do)]
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    op = torch.empty_like(dev[0])
+    lse = torch.empty((B, nh, N), dtype=torch.float32, device="cuda")
+    lib.dfs_get_error_flags(clear=True)
+    lib.dfs_sparse_attn_fwd(s, dev[0], dev[1], dev[2], it, ct, kcap, 0.0, op, lse)
+    grads = [torch.empty_like(dev[0]) for _ in range(3)]
+    ws = torch.empty(lib.dfs_workspace_bytes(s, lib.DFS_WS_ATTN_BWD), dtype=torch.uint8, device="cuda")
+    lib.dfs_sparse_attn_bwd(s, dev[0], dev[1], dev[2], op, dev[3], lse, it, ct, kcap, 0.0, *grads, ws)
+    torch.cuda.synchronize()
+    flags = lib.dfs_get_error_flags(clear=True)
+    assert flags & lib.DFS_FLAG_BAD_KV_INDEX
+    assert not flags & lib.DFS_FLAG_WAIT_TIMEOUT
+    got = [g.float().cpu().numpy() for g in grads]
+    ref = attention.block_sparse_attention_bwd(*(t.double().numpy() for t in (q, k, v, do)), clean_idx, clean_cnt,
+                                               128)
+    _check(got, ref, "invalid entries")
+    # The backward over the clean lists, from the same forward outputs, is
+    # bitwise the same. (The forward's own results may differ by rounding:
+    # a split last-wave CTA halves the counted list, invalid entries included.)
+    ic, cc = torch.from_numpy(clean_idx).cuda(), torch.from_numpy(clean_cnt).cuda()
+    grads2 = [torch.empty_like(dev[0]) for _ in range(3)]
+    lib.dfs_sparse_attn_bwd(s, dev[0], dev[1], dev[2], op, dev[3], lse, ic, cc, kcap, 0.0, *grads2, ws)
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == 0
+    for x, y in zip(grads, grads2):
+        assert torch.equal(x, y)
+
+
 def test_full_mask_matches_dense_gradients(lib):
     B, nh, D, N = 1, 2, 64, 640
     nb = N // 128
