@@ -231,8 +231,12 @@ int dfs_select_mask(const dfs_shape *shape, const float *scores, const dfs_selec
  * sum of exp of the scaled logits. scale <= 0 selects 1/sqrt(D).
  * The softmax runs in fp32, P is rounded to bf16 for the P.V product,
  * accumulation is fp32. Indices outside [0, nb) are skipped and set
- * DFS_FLAG_BAD_KV_INDEX. Every device wait is bounded; a wait that gives up
- * sets DFS_FLAG_WAIT_TIMEOUT and the kernel returns early.                */
+ * DFS_FLAG_BAD_KV_INDEX. The two lists a CTA works on are staged in shared
+ * memory beside the tiles: for D = 128 and blk = 128, min(kcap, nb) may be
+ * at most 4202 (a little over half that with frame-exact masking); a longer
+ * list returns DFS_ERR_UNSUPPORTED before anything is launched. Every
+ * device wait is bounded; a wait that gives up sets DFS_FLAG_WAIT_TIMEOUT
+ * and the kernel returns early.                                           */
 int dfs_sparse_attn_fwd(const dfs_shape *shape, const void *qp, const void *kp, const void *vp,
                         const int32_t *kv_idx, const int32_t *kv_cnt, int kcap, float scale,
                         void *op, float *lse, dfs_stream_t stream);

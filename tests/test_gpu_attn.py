@@ -304,6 +304,34 @@ def test_binding_rejects_wrong_tensors(lib):
     assert bool((op == 7.0).all())
 
 
+def test_list_length_limit(lib):
+    """The two lists of a CTA are staged in shared memory: for D = 128 and
+    blk = 128, min(kcap, nb) = 4202 still fits (232,448 bytes) and 4203 is
+    rejected with DFS_ERR_UNSUPPORTED before anything is launched. All
+    tensors are sized for the shape, so a regression fails the assertion
+    rather than touching memory it does not own."""
+    D, nb = 128, 4203
+    N = nb * 128
+    s = lib.Shape(1, 1, D, 1, 1, N, 128, 16)
+    q = torch.zeros((1, 1, N, D), dtype=torch.bfloat16, device="cuda")
+    cnt = torch.zeros((1, 1, nb), dtype=torch.int32, device="cuda")      # empty lists
+    for kcap, ok in ((4202, True), (4203, False)):
+        idx = torch.zeros((1, 1, nb, kcap), dtype=torch.int32, device="cuda")
+        op = torch.full((1, 1, N, D), 7.0, dtype=torch.bfloat16, device="cuda")
+        if ok:
+            lib.dfs_sparse_attn_fwd(s, q, q, q, idx, cnt, kcap, 0.0, op)
+            torch.cuda.synchronize()
+            assert lib.dfs_get_error_flags(clear=True) == 0
+            assert bool((op == 0).all())                    # rows with no kept block
+        else:
+            with pytest.raises(lib.DfsError) as e:
+                lib.dfs_sparse_attn_fwd(s, q, q, q, idx, cnt, kcap, 0.0, op)
+            assert e.value.status == lib.DFS_ERR_UNSUPPORTED
+            torch.cuda.synchronize()
+            assert bool((op == 7.0).all())
+        del idx, op
+
+
 def _per_head_order(cnt, kmax):
     """The rows of each head stably sorted by clamped count, largest first;
     heads in order (flat row indices)."""
