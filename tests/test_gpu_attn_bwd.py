@@ -169,6 +169,60 @@ def test_invalid_entries_are_skipped_and_flagged(lib):
         assert torch.equal(x, y)
 
 
+def test_maximum_block_count(lib):
+    """nb = 8192, the largest the backward takes (1,048,576 tokens at D = 64),
+    runs and is right; 8193 is rejected before anything is launched. Query
+    block I keeps blocks {0, I}, so key block J >= 1 is kept by query block J
+    alone and key block 0 by all 8192 (one dK/dV CTA walks the whole
+    transposed list): dQ of query block J and dK, dV of key block J equal
+    those of the two-block problem (blocks 0 and J) in the oracle."""
+    D, blk = 64, 128
+    nb_max = 8192
+    N_big = (nb_max + 1) * blk
+    N = nb_max * blk
+    g = torch.Generator().manual_seed(31)
+    host = [(torch.randn((1, 1, N_big, D), generator=g) * 1.3).to(torch.bfloat16) for _ in range(3)]
+    host.append((torch.randn((1, 1, N_big, D), generator=g) * 0.5).to(torch.bfloat16))
+    dev = [t.cuda() for t in host]
+    view = [t[:, :, :N] for t in dev]                        # contiguous: leading dims are 1
+    s = lib.Shape(1, 1, D, 1, 1, N, blk, 16)
+    idx = np.zeros((1, 1, nb_max, 2), dtype=np.int32)
+    idx[0, 0, :, 1] = np.arange(nb_max)
+    cnt = np.full((1, 1, nb_max), 2, dtype=np.int32)
+    cnt[0, 0, 0] = 1                                         # block 0 keeps only itself
+    it, ct = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    op = torch.empty_like(view[0])
+    lse = torch.empty((1, 1, N), dtype=torch.float32, device="cuda")
+    lib.dfs_get_error_flags(clear=True)
+    lib.dfs_sparse_attn_fwd(s, view[0], view[1], view[2], it, ct, 2, 0.0, op, lse)
+    grads = [torch.empty_like(view[0]) for _ in range(3)]
+    ws = torch.empty(lib.dfs_workspace_bytes(s, lib.DFS_WS_ATTN_BWD), dtype=torch.uint8, device="cuda")
+    lib.dfs_sparse_attn_bwd(s, view[0], view[1], view[2], op, view[3], lse, it, ct, 2, 0.0, *grads, ws)
+    torch.cuda.synchronize()
+    assert lib.dfs_get_error_flags(clear=True) == 0
+    for J in (1, 2, 4095, nb_max - 1):
+        rows = np.r_[0:blk, J * blk:(J + 1) * blk]
+        mini = [t[:, :, rows].double().numpy() for t in host]
+        mi = np.array([[[[0, -1], [0, 1]]]], dtype=np.int32)
+        mc = np.array([[[1, 2]]], dtype=np.int32)
+        ref = attention.block_sparse_attention_bwd(*mini, mi, mc, blk, rows=[(0, 0, 1)])
+        sl = slice(J * blk, (J + 1) * blk)
+        got = [x[:, :, sl].float().cpu().numpy() for x in grads]
+        _check(got, [r[:, :, blk:] for r in ref], f"nb 8192, block {J}")
+    # one more block than the backward takes: rejected on the host side of the launch
+    s2 = lib.Shape(1, 1, D, 1, 1, N_big, blk, 16)
+    idx2 = torch.zeros((1, 1, nb_max + 1, 2), dtype=torch.int32, device="cuda")
+    cnt2 = torch.ones((1, 1, nb_max + 1), dtype=torch.int32, device="cuda")
+    lse2 = torch.zeros((1, 1, N_big), dtype=torch.float32, device="cuda")
+    out2 = [torch.full_like(dev[0], 3.0) for _ in range(3)]
+    ws2 = torch.empty(lib.dfs_workspace_bytes(s2, lib.DFS_WS_ATTN_BWD), dtype=torch.uint8, device="cuda")
+    with pytest.raises(lib.DfsError) as e:
+        lib.dfs_sparse_attn_bwd(s2, dev[0], dev[1], dev[2], dev[0], dev[3], lse2, idx2, cnt2, 2, 0.0, *out2, ws2)
+    assert e.value.status == lib.DFS_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert all(bool((x == 3.0).all()) for x in out2)
+
+
 def test_full_mask_matches_dense_gradients(lib):
     B, nh, D, N = 1, 2, 64, 640
     nb = N // 128
