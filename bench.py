@@ -50,8 +50,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch from one ncu capture of
 # that workload, valid only for the attention sources
 # whose hash is recorded with it; reported as null once they change.
-ATTN_TRAFFIC = {"wan_1p3b_layer": (298_866_176 + 83_991_552, "055f4a481e84b06c"),
-                "hunyuan_layer": (4_869_139_712 + 798_416_896, "055f4a481e84b06c")}
+ATTN_TRAFFIC = {"wan_1p3b_layer": (298_117_376 + 81_682_176, "66a54f472c7b2e82"),
+                "hunyuan_layer": (4_672_438_528 + 755_917_056, "66a54f472c7b2e82")}
 ATTN_SOURCES = ("attn.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh", "lvsa.cuh", "tmap.cuh")
 
 

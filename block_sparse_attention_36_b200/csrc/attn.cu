@@ -66,6 +66,15 @@ constexpr long long kWaitLimit = 4000000000ll;   // per pipeline wait
 constexpr long long kDrainLimit = 2000000000ll;  // per drain wait
 constexpr int kRing = 4;                           // K/V ring stages
 constexpr int kThreads = 384;                      // 3 warpgroups
+// Warp-specialised register split of the 512-column (blk 128) kernels, which
+// are launched at the 168-register cap of 384 threads: warpgroup 0
+// (producer, MMA issuer, list warps) gives registers back and the two
+// softmax warpgroups take them (setmaxnreg), which removes the softmax's
+// spills. 128 * 80 + 256 * 208 = 63,488 <= 384 * 168 = 64,512 registers;
+// the launch checks the kernel's register count against this before it
+// runs (an increase beyond the block's registers would never complete).
+constexpr int kRegWg0 = 80;
+constexpr int kRegSoftmax = 208;
 constexpr int kQRows = 128;                        // MMA M
 
 template <int D, int BLK>
@@ -289,6 +298,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int n[2] = {bars->n_kv[0], bars->n_kv[1]};
   const int jmax = max(n[0], n[1]);
   if (warp < 4) {
+  if (BLK == 128) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegWg0) : "memory");
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Warp-uniform loop; elect.sync picks the lane that arms a barrier or
@@ -403,6 +413,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   } else {
     // ------------------------------------------------------------ softmax
+    if (BLK == 128) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax) : "memory");
     const int x = warp < 8 ? 0 : 1;                 // slot
     const int I = slot_I(x);
     const int bh = slot_bh(x);
@@ -682,6 +693,13 @@ int launch_attn(const dfs::Dims& d, const void* qp, const void* kp, const void* 
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, BLK, EMU, FRAME>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return DFS_ERR_CUDA;
+  if (BLK == 128) {
+    // the register split must fit the registers the CTA is launched with
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, BLK, EMU, FRAME>) != cudaSuccess) return DFS_ERR_CUDA;
+    const int launched = ((fa.numRegs + 7) / 8) * 8;
+    if (128 * kRegWg0 + 256 * kRegSoftmax > launched * kThreads) return DFS_ERR_UNSUPPORTED;
+  }
   // virtual rows (see OutMap), two-row CTAs, and the split of the last wave
   const long long V = om.order ? om.rows : 2LL * d.BH * ((d.nb + 1) / 2);
   const long long pairs = (V + 1) / 2;
